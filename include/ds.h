@@ -1,0 +1,201 @@
+/*
+ * ds.h -- C ABI of the token-sparse decode-attention library (libds.so).
+ *
+ * Method: "Post-Training Sparse Attention with Double Sparsity" (arXiv
+ * 2408.07092).  A static set of important feature channels per head (channel
+ * sparsity, fixed offline: Method details, Core idea / Technical framework)
+ * is used to score every cached token cheaply; the tokens with the highest
+ * scores are kept (Method details, Key design); exact softmax attention then
+ * runs over the kept tokens only (token sparsity: Abstract, Key points 2).
+ *
+ * Notation (one decode step, one query token per sequence):
+ *   B      sequences in the batch
+ *   Hq     query heads; Hkv KV heads; Hq % Hkv == 0; query head h reads
+ *          KV head g(h) = h / (Hq / Hkv)
+ *   d      head dimension; this build supports d == 128 only
+ *   T_cap  token capacity of the K/V and label caches; T <= T_cap tokens valid
+ *   r      label channels per query head (1 <= r <= d)
+ *   k      tokens kept per query head (1 <= k <= T)
+ *
+ * Layouts (row-major, contiguous, element type in brackets):
+ *   Q      [B, Hq, d]            (bf16)
+ *   K, V   [B, Hkv, T_cap, d]    (bf16)   one 256-byte row per token
+ *   C      [Hq, r]               (int32)  channel ids in [0, d), ascending
+ *                                         by convention (any order works)
+ *   label  [B, Hq, T_cap, r]     (bf16)   label[b,h,t,j] = K[b,g(h),t,C[h,j]]
+ *   scores [B*Hq, T]             (fp32)
+ *   idx    [B*Hq, k]             (int32)  ascending token ids
+ *   O      [B, Hq, d]            (fp32)
+ *   lse    [B, Hq]               (fp32)   natural log of the softmax
+ *                                         denominator, including the scale
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or synchronises.  Every pointer must be 16-byte
+ *     aligned.  Calls are asynchronous on `stream` (0 = legacy default).
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns DS_ERR_INVALID_ARG (or DS_ERR_UNSUPPORTED for a valid
+ *     but unimplemented shape) and launches nothing.
+ *   - Device-side values the host cannot see cheaply (channel ids, token
+ *     indices) are masked or clamped into range inside the kernels so that no
+ *     access leaves its buffer; each such event sets a bit in a per-device
+ *     status word read by ds_device_status().  Kernels never trap.
+ *   - A launch failure returns DS_ERR_CUDA (details: ds_last_cuda_error()).
+ *   - Calls on different streams may run concurrently if their outputs and
+ *     workspaces do not overlap.
+ */
+#ifndef POST_TOKEN_SPARSE_DS_H_
+#define POST_TOKEN_SPARSE_DS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same opaque handle as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st* ds_stream_t;
+
+typedef enum {
+  DS_OK = 0,
+  DS_ERR_INVALID_ARG = 1, /* null/misaligned pointer, out-of-range size     */
+  DS_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d != 128)      */
+  DS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required     */
+  DS_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed    */
+} ds_status;
+
+typedef struct {
+  int32_t B, Hq, Hkv, d, T_cap, r;
+} ds_dims;
+
+/* Operation ids for ds_workspace_size(). */
+enum {
+  DS_OP_LABEL_APPEND = 0,
+  DS_OP_SCORE = 1,
+  DS_OP_TOPK = 2,
+  DS_OP_SPARSE_DECODE = 3,
+  DS_OP_DECODE = 4,
+  DS_OP_SCORE_TOPK = 5
+};
+
+/* Device status bits (ds_device_status). */
+enum {
+  DS_DEV_BAD_CHANNEL = 1u, /* a channel id in C was outside [0, d); masked  */
+  DS_DEV_BAD_INDEX = 2u    /* a token index was outside [0, T); clamped     */
+};
+
+/*
+ * ds_label_append -- build or extend the label cache.
+ *
+ * label[b,h,t,j] = K[b, g(h), t, C[h,j]] for every b, h, j and
+ * t0 <= t < t0 + n.  The label cache is the contiguous copy of each query
+ * head's r calibrated channels of K (channel sparsity; Double Sparsity page,
+ * Method details: Core idea and Technical framework -- the channel pattern is
+ * static, so it is found offline and applied at run time).  Call once over
+ * the prompt (t0 = 0, n = T) and once per generated token (t0 = T-1, n = 1).
+ *
+ * K: [B,Hkv,T_cap,d] bf16.  C: [Hq,r] int32.  label: [B,Hq,T_cap,r] bf16,
+ * written only in rows [t0, t0+n).  Requires 0 <= t0, 1 <= n,
+ * t0 + n <= T_cap.  Bit-exact copy: no arithmetic.
+ */
+ds_status ds_label_append(const void* K, const int32_t* C, void* label, ds_dims dims,
+                          int32_t t0, int32_t n, ds_stream_t stream);
+
+/*
+ * ds_score -- approximate (channel-sparse) attention scores.
+ *
+ * scores[b*Hq+h, t] = sum_j q[b,h,C[h,j]] * label[b,h,t,j] for t < T,
+ * unscaled, products and sums in fp32.  The tokens with the higher values of
+ * this score are the important ones (Double Sparsity page, Method details:
+ * Key design).
+ *
+ * Q: [B,Hq,d] bf16.  C: [Hq,r] int32.  label: [B,Hq,T_cap,r] bf16.
+ * scores: [B*Hq, T] fp32.  Requires 1 <= T <= T_cap.
+ */
+ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* scores,
+                   ds_dims dims, int32_t T, ds_stream_t stream);
+
+/*
+ * ds_topk -- per-row top-k token indices.
+ *
+ * For each of the BH rows of `scores` ([BH, T] fp32), writes to idx ([BH, k]
+ * int32) the k indices with the largest scores, ascending.  Ties go to the
+ * lower index; -0.0 and +0.0 are equal; +-inf order normally; NaN is outside
+ * the contract (no fault, unspecified choice).  Token selection by the higher
+ * activation (Double Sparsity page, Method details: Key design).
+ *
+ * Requires 1 <= k <= T <= 655360 and BH <= 65535.  Needs no workspace
+ * (ds_workspace_size returns 0); `ws` may be NULL.
+ */
+ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int32_t k,
+                  void* ws, size_t ws_bytes, ds_stream_t stream);
+
+/*
+ * ds_score_topk -- ds_score followed by ds_topk in one launch.
+ *
+ * Same results as the two calls (same fp32 scores, same index set), without
+ * writing the scores to memory unless `scores` is non-NULL.  Limits as for
+ * ds_topk.  Needs no workspace.
+ */
+ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
+                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream);
+
+/*
+ * ds_sparse_decode -- exact softmax attention over the selected tokens.
+ *
+ * For each (b, h) with rows i = idx[b*Hq+h, 0..k):
+ *   l_i = scale * (q[b,h,:] . K[b,g(h),i,:]);  w = softmax(l);
+ *   O[b,h,:] = sum_i w_i V[b,g(h),i,:];  lse[b,h] = log sum_i exp(l_i).
+ * Self-attention computed with the important tokens only (Double Sparsity
+ * page, Abstract; Key points 2).  The k rows are split into chunks processed
+ * in parallel; each chunk keeps a running max and sum and the chunks are
+ * combined by log-sum-exp weights.  fp32 accumulation.
+ *
+ * Q: [B,Hq,d] bf16; K, V: [B,Hkv,T_cap,d] bf16; idx: [B*Hq,k] int32 with
+ * entries in [0, T) (out-of-range entries are clamped and flagged);
+ * O: [B,Hq,d] fp32; lse: [B,Hq] fp32 or NULL.  Requires 1 <= k <= T <= T_cap.
+ * ws: ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k) bytes of device
+ * memory (contents need not be initialised; may be NULL when that size is 0).
+ */
+ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
+                           float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
+                           void* ws, size_t ws_bytes, ds_stream_t stream);
+
+/*
+ * ds_decode -- dense decode attention over all T cached tokens: the operation
+ * token sparsity accelerates (Double Sparsity page, Experimental highlights:
+ * attention-operation speed-up).  Same as ds_sparse_decode with
+ * idx = 0..T-1 for every head.  ws: ds_workspace_size(DS_OP_DECODE, dims, T,
+ * T) bytes.
+ */
+ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float* lse,
+                    ds_dims dims, int32_t T, float scale, void* ws, size_t ws_bytes,
+                    ds_stream_t stream);
+
+/*
+ * Bytes of device workspace `op` needs for these sizes (0 if none).  Depends
+ * only on the arguments, never on the device.  Returns 0 for invalid sizes.
+ */
+size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k);
+
+/* Human-readable name of a status code (static storage). */
+const char* ds_status_string(ds_status s);
+
+/* Text of the last CUDA error seen by this library on the calling thread. */
+const char* ds_last_cuda_error(void);
+
+/*
+ * Reads (and, if `clear` != 0, resets) the status bits that kernels set on
+ * the current device (DS_DEV_*).  Synchronises `stream` first.
+ */
+ds_status ds_device_status(uint32_t* bits, int32_t clear, ds_stream_t stream);
+
+/* Number of kernels this library has launched in this process (host count). */
+uint64_t ds_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POST_TOKEN_SPARSE_DS_H_ */

@@ -1,0 +1,215 @@
+"""Token-sparse (Double-Sparsity-style) decode attention on B200 (sm_100a).
+
+Thin Python binding of ``libds.so`` (C ABI in ``include/ds.h``): argument
+marshalling only.  Every step of the decode path runs in the library's CUDA
+kernels; PyTorch supplies device memory and the current stream.  Importing
+this package fails if the compiled library is missing -- there is no CPU or
+PyTorch fallback.  Build it with ``python -m post_token_sparse_b200.build``.
+
+Calls mirror the C ABI:
+
+    label_append(K, C, label, t0, n)            label cache rows [t0, t0+n)
+    score(Q, C, label, scores, T)               channel-sparse scores
+    topk(scores, idx)                           per-row top-k, ascending
+    score_topk(Q, C, label, idx, T, scores=None)  the two above in one launch
+    sparse_decode(Q, K, V, idx, O, T, scale, lse=None, ws=None)
+    decode(Q, K, V, O, T, scale, lse=None, ws=None)   dense reference
+
+All tensors must be CUDA, contiguous, with the dtypes and shapes of
+``include/ds.h``; the C library checks sizes and alignment and raises
+``DsError`` with its status name on any failure.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libds.so")
+
+DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
+OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK = range(6)
+DEV_BAD_CHANNEL, DEV_BAD_INDEX = 1, 2
+
+
+class DsError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        name = _lib.ds_status_string(status).decode()
+        detail = ""
+        if status == DS_ERR_CUDA:
+            detail = ": " + _lib.ds_last_cuda_error().decode()
+        super().__init__(f"{what} failed with {name}{detail}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("T_cap", ctypes.c_int32), ("r", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "Dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m post_token_sparse_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, u32p = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)
+    st = ctypes.c_int
+    sig = {
+        "ds_label_append": [vp, vp, vp, Dims, i32, i32, vp],
+        "ds_score": [vp, vp, vp, vp, Dims, i32, vp],
+        "ds_topk": [vp, vp, i32, i32, i32, vp, ctypes.c_size_t, vp],
+        "ds_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
+        "ds_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, vp,
+                             ctypes.c_size_t, vp],
+        "ds_decode": [vp, vp, vp, vp, vp, Dims, i32, ctypes.c_float, vp, ctypes.c_size_t, vp],
+        "ds_device_status": [u32p, i32, vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = st
+    lib.ds_workspace_size.argtypes = [i32, Dims, i32, i32]
+    lib.ds_workspace_size.restype = ctypes.c_size_t
+    lib.ds_status_string.argtypes = [st]
+    lib.ds_status_string.restype = ctypes.c_char_p
+    lib.ds_last_cuda_error.argtypes = []
+    lib.ds_last_cuda_error.restype = ctypes.c_char_p
+    lib.ds_kernel_launches.argtypes = []
+    lib.ds_kernel_launches.restype = ctypes.c_uint64
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    """The loaded ctypes library (for callers that want the raw C ABI)."""
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise TypeError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != DS_OK:
+        raise DsError(status, what)
+
+
+def dims_of(Q: torch.Tensor, K: torch.Tensor, r: int) -> Dims:
+    """Dims from Q [B,Hq,d] and K [B,Hkv,T_cap,d]."""
+    B, Hq, d = Q.shape
+    _, Hkv, T_cap, _ = K.shape
+    return Dims(B, Hq, Hkv, d, T_cap, r)
+
+
+def workspace_size(op: int, dims: Dims, T: int, k: int) -> int:
+    return int(_lib.ds_workspace_size(op, dims, T, k))
+
+
+def workspace(op: int, dims: Dims, T: int, k: int, device) -> torch.Tensor | None:
+    """A device buffer of the size ``op`` needs (None when it needs none)."""
+    n = workspace_size(op, dims, T, k)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+# ---------------------------------------------------------------------------
+# the calls
+
+def label_append(K, C, label, t0: int, n: int):
+    B, Hkv, T_cap, d = K.shape
+    Hq, r = C.shape
+    dims = Dims(B, Hq, Hkv, d, T_cap, r)
+    _check(_lib.ds_label_append(_ptr(K, torch.bfloat16, "K"), _ptr(C, torch.int32, "C"),
+                                _ptr(label, torch.bfloat16, "label"), dims, t0, n,
+                                _stream(K.device)), "ds_label_append")
+
+
+def score(Q, C, label, scores, T: int):
+    B, Hq, d = Q.shape
+    _, _, T_cap, r = label.shape
+    dims = Dims(B, Hq, Hq, d, T_cap, r)  # the score step does not read K
+    _check(_lib.ds_score(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
+                         _ptr(label, torch.bfloat16, "label"), _ptr(scores, torch.float32,
+                                                                     "scores"),
+                         dims, T, _stream(Q.device)), "ds_score")
+
+
+def topk(scores, idx):
+    BH, T = scores.shape
+    k = idx.shape[-1]
+    if idx.numel() != BH * k:
+        raise TypeError("idx must have BH*k elements")
+    _check(_lib.ds_topk(_ptr(scores, torch.float32, "scores"), _ptr(idx, torch.int32, "idx"),
+                        BH, T, k, None, 0, _stream(scores.device)), "ds_topk")
+
+
+def score_topk(Q, C, label, idx, T: int, scores=None):
+    B, Hq, d = Q.shape
+    _, _, T_cap, r = label.shape
+    dims = Dims(B, Hq, Hq, d, T_cap, r)
+    k = idx.shape[-1]
+    _check(_lib.ds_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
+                              _ptr(label, torch.bfloat16, "label"),
+                              _ptr(scores, torch.float32, "scores"),
+                              _ptr(idx, torch.int32, "idx"), dims, T, k, _stream(Q.device)),
+           "ds_score_topk")
+
+
+def sparse_decode(Q, K, V, idx, O, T: int, scale: float, lse=None, ws=None):
+    dims = dims_of(Q, K, 1)
+    k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_SPARSE_DECODE, dims, T, k, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_sparse_decode(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+                                 _ptr(V, torch.bfloat16, "V"), _ptr(idx, torch.int32, "idx"),
+                                 _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"),
+                                 dims, T, k, scale, _ptr(ws, None, "ws"), nbytes,
+                                 _stream(Q.device)), "ds_sparse_decode")
+
+
+def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):
+    dims = dims_of(Q, K, 1)
+    if ws is None:
+        ws = workspace(OP_DECODE, dims, T, T, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_decode(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+                          _ptr(V, torch.bfloat16, "V"), _ptr(O, torch.float32, "O"),
+                          _ptr(lse, torch.float32, "lse"), dims, T, scale,
+                          _ptr(ws, None, "ws"), nbytes, _stream(Q.device)), "ds_decode")
+
+
+def device_status(clear: bool = True, device=None) -> int:
+    """Status bits kernels set on the current device (DEV_BAD_CHANNEL, DEV_BAD_INDEX)."""
+    bits = ctypes.c_uint32(0)
+    _check(_lib.ds_device_status(ctypes.byref(bits), int(clear), _stream(device)),
+           "ds_device_status")
+    return int(bits.value)
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libds.so in this process so far."""
+    return int(_lib.ds_kernel_launches())

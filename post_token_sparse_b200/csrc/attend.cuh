@@ -1,0 +1,260 @@
+// Decode attention over a set of K/V rows: the selected tokens (sparse) or all
+// T tokens (dense).
+//
+// Token sparsity (Double Sparsity, Abstract; Key points 2): exact softmax
+// attention computed over the important tokens only.  HBM-bound: every
+// selected row is 256 B of K plus 256 B of V, read once.
+//
+// Grid (G, S, B*Hkv): the G query heads sharing one KV head are neighbours in
+// launch order (their dense K/V reads meet in L2), and each head's rows are
+// cut into S splits.  A CTA has kAttnWarps warps; every warp owns a
+// contiguous run of its split's rows and walks it 4 rows per step.  Lane
+// (g = lane/8, c = lane%8) handles row g of the step and the 16-byte chunks c
+// and c+8 of that row (dims 8c..8c+7 and 64+8c..64+8c+7) of both K and V.
+//
+// Staging: each lane copies exactly the bytes it later reads with cp.async
+// into a per-warp ring of kAttnStages steps, so the pipeline needs neither
+// block barriers nor cross-lane hand-off: cp.async.wait_group is the only
+// wait.  Per row: 16 FMAs + 3 xor-shuffles for the logit, an online-softmax
+// update (running max m, sum l, log2 domain), 16 FMAs into the accumulator.
+// Warps then merge through shared memory; with S > 1 each split writes
+// (m, l, unnormalised o) and k_lse_merge combines them.
+#pragma once
+
+#include "common.cuh"
+
+namespace ds {
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnThreads = kAttnWarps * 32;
+constexpr int kAttnStages = 8;
+constexpr int kAttnStageU4 = 4 * 32;  // 4 rows x (16 uint4 of K + 16 uint4 of V) = 2 KB
+constexpr int kPartialStride = 132;   // floats per split partial: m, l, pad, pad, o[128]
+constexpr int kMaxRowsPerSplitSparse = 2048;
+
+struct AttnParams {
+  const uint16_t* Q;
+  const uint16_t* K;
+  const uint16_t* V;
+  const int32_t* idx;  // null: dense (rows 0..T-1)
+  float* O;
+  float* lse;      // optional
+  float* partial;  // [BH, S, kPartialStride] when S > 1
+  int Hq, Hkv, T_cap, T;
+  int rows;           // k (sparse) or T (dense)
+  int rows_per_split; // multiple of 4
+  float scale_log2;   // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ float dot8(const uint4& v, const float* q) {
+  float a = bf_lo(v.x) * q[0];
+  a = fmaf(bf_hi(v.x), q[1], a);
+  a = fmaf(bf_lo(v.y), q[2], a);
+  a = fmaf(bf_hi(v.y), q[3], a);
+  a = fmaf(bf_lo(v.z), q[4], a);
+  a = fmaf(bf_hi(v.z), q[5], a);
+  a = fmaf(bf_lo(v.w), q[6], a);
+  a = fmaf(bf_hi(v.w), q[7], a);
+  return a;
+}
+
+__device__ __forceinline__ void axpy8(float* acc, float a, float p, const uint4& v) {
+  acc[0] = fmaf(acc[0], a, p * bf_lo(v.x));
+  acc[1] = fmaf(acc[1], a, p * bf_hi(v.x));
+  acc[2] = fmaf(acc[2], a, p * bf_lo(v.y));
+  acc[3] = fmaf(acc[3], a, p * bf_hi(v.y));
+  acc[4] = fmaf(acc[4], a, p * bf_lo(v.z));
+  acc[5] = fmaf(acc[5], a, p * bf_hi(v.z));
+  acc[6] = fmaf(acc[6], a, p * bf_lo(v.w));
+  acc[7] = fmaf(acc[7], a, p * bf_hi(v.w));
+}
+
+// weight of a partial with running max m against a common max mn (0 if empty)
+__device__ __forceinline__ float rescale(float m, float mn) {
+  return m == -INFINITY ? 0.f : exp2f(m - mn);
+}
+
+template <bool kSparse>
+__global__ void __launch_bounds__(kAttnThreads)
+k_attend(const AttnParams p) {
+  extern __shared__ __align__(16) uint4 smem_u4[];
+  uint4* ring = smem_u4;                                                 // [warps][stages][128]
+  float* red = reinterpret_cast<float*>(ring + kAttnWarps * kAttnStages * kAttnStageU4);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(red + kAttnWarps * 132);   // [rows_per_split]
+
+  const int G = p.Hq / p.Hkv;
+  const int bkv = blockIdx.z;  // b * Hkv + g
+  const int b = bkv / p.Hkv;
+  const int h = (bkv % p.Hkv) * G + blockIdx.x;
+  const int bh = b * p.Hq + h;
+  const int S = gridDim.y, split = blockIdx.y;
+  const int r0 = split * p.rows_per_split;
+  const int nrows = min(p.rows_per_split, p.rows - r0);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 3, c = lane & 7;
+
+  if constexpr (kSparse) {
+    const int32_t* src = p.idx + (size_t)bh * p.rows + r0;
+    for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
+      int t = src[i];
+      if (t < 0 || t >= p.T) {
+        flag_status(2u);
+        t = min(max(t, 0), p.T - 1);
+      }
+      idx_s[i] = t;
+    }
+    __syncthreads();
+  }
+
+  // this lane's 16 query values, pre-scaled into the log2 domain
+  float q[16];
+  {
+    const uint4* qrow = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim);
+    const uint4 a = qrow[c], bq = qrow[8 + c];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q[2 * i] = bf_lo(w[i]) * p.scale_log2;
+      q[2 * i + 1] = bf_hi(w[i]) * p.scale_log2;
+    }
+  }
+
+  // rows of this warp: [w_begin, w_end) relative to r0
+  const int rpw = ((nrows + kAttnWarps - 1) / kAttnWarps + 3) & ~3;
+  const int w_begin = min(warp * rpw, nrows);
+  const int w_end = min(w_begin + rpw, nrows);
+  const int nsteps = (w_end - w_begin + 3) >> 2;
+
+  const size_t kv_base = (size_t)bkv * p.T_cap * kHeadDim;
+  const uint16_t* Kh = p.K + kv_base;
+  const uint16_t* Vh = p.V + kv_base;
+  uint4* my_ring = ring + warp * kAttnStages * kAttnStageU4;
+
+  auto issue = [&](int step) {
+    const int lr = w_begin + step * 4 + g;  // row within the split
+    if (lr < w_end) {
+      const int t = kSparse ? idx_s[lr] : r0 + lr;
+      const uint4* krow = reinterpret_cast<const uint4*>(Kh + (size_t)t * kHeadDim);
+      const uint4* vrow = reinterpret_cast<const uint4*>(Vh + (size_t)t * kHeadDim);
+      uint4* st = my_ring + (step % kAttnStages) * kAttnStageU4 + g * 32;
+      cp_async16(st + c, krow + c);
+      cp_async16(st + 8 + c, krow + 8 + c);
+      cp_async16(st + 16 + c, vrow + c);
+      cp_async16(st + 24 + c, vrow + 8 + c);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < kAttnStages - 1; ++s) {
+    if (s < nsteps) issue(s);
+    cp_async_commit();
+  }
+
+  float m = -INFINITY, l = 0.f;
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+
+  for (int n = 0; n < nsteps; ++n) {
+    if (n + kAttnStages - 1 < nsteps) issue(n + kAttnStages - 1);
+    cp_async_commit();
+    cp_async_wait<kAttnStages - 1>();
+
+    const uint4* st = my_ring + (n % kAttnStages) * kAttnStageU4 + g * 32;
+    const uint4 klo = st[c], khi = st[8 + c];
+    float x = dot8(klo, q) + dot8(khi, q + 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    if (w_begin + n * 4 + g < w_end) {
+      float a = 1.f;
+      if (x > m) {
+        a = exp2f(m - x);  // 0 when m is still -inf
+        l *= a;
+        m = x;
+      }
+      const float pw = exp2f(x - m);
+      l += pw;
+      const uint4 vlo = st[16 + c], vhi = st[24 + c];
+      axpy8(acc, a, pw, vlo);
+      axpy8(acc + 8, a, pw, vhi);
+    }
+  }
+  cp_async_wait<0>();
+
+  // merge the four row slots of the warp (lanes with equal c)
+#pragma unroll
+  for (int o = 8; o <= 16; o <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+    const float mn = fmaxf(m, m2);
+    const float a1 = rescale(m, mn), a2 = rescale(m2, mn);
+    l = l * a1 + l2 * a2;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, acc[i], o);
+      acc[i] = acc[i] * a1 + other * a2;
+    }
+    m = mn;
+  }
+  // warp partials -> shared memory: red[w*132 + {0: m, 1: l, 4..131: o}]
+  float* wr = red + warp * 132;
+  if (g == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      wr[4 + c * 8 + i] = acc[i];
+      wr[4 + 64 + c * 8 + i] = acc[8 + i];
+    }
+    if (c == 0) {
+      wr[0] = m;
+      wr[1] = l;
+    }
+  }
+  __syncthreads();
+
+  // thread j merges dim j over the warps
+  const int j = threadIdx.x;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, red[w * 132]);
+  float L = 0.f, o = 0.f;
+#pragma unroll
+  for (int w = 0; w < kAttnWarps; ++w) {
+    const float a = rescale(red[w * 132], M);
+    L = fmaf(red[w * 132 + 1], a, L);
+    o = fmaf(red[w * 132 + 4 + j], a, o);
+  }
+  if (S == 1) {
+    p.O[(size_t)bh * kHeadDim + j] = o / L;
+    if (p.lse && j == 0) p.lse[bh] = (M + log2f(L)) * 0.69314718055994530942f;
+  } else {
+    float* part = p.partial + ((size_t)bh * S + split) * kPartialStride;
+    part[4 + j] = o;
+    if (j == 0) {
+      part[0] = M;
+      part[1] = L;
+    }
+  }
+}
+
+// Combine S split partials per head: O = sum_s 2^(m_s-M) o_s / sum_s 2^(m_s-M) l_s.
+// grid BH, block 128 (thread j = dim j).
+__global__ void __launch_bounds__(kHeadDim)
+k_lse_merge(const float* __restrict__ partial, float* __restrict__ O, float* __restrict__ lse,
+            int S) {
+  const int bh = blockIdx.x, j = threadIdx.x;
+  const float* part = partial + (size_t)bh * S * kPartialStride;
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, part[s * kPartialStride]);
+  float L = 0.f, o = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float a = rescale(part[s * kPartialStride], M);
+    L = fmaf(part[s * kPartialStride + 1], a, L);
+    o = fmaf(part[s * kPartialStride + 4 + j], a, o);
+  }
+  O[(size_t)bh * kHeadDim + j] = o / L;
+  if (lse && j == 0) lse[bh] = (M + log2f(L)) * 0.69314718055994530942f;
+}
+
+}  // namespace ds

@@ -1,0 +1,400 @@
+// C ABI of libds.so: argument checks, launch configuration and launches.
+//
+// All kernels live in this one translation unit (no relocatable device code).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "ds.h"
+
+#include "attend.cuh"
+#include "common.cuh"
+#include "label.cuh"
+#include "score.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using namespace ds;
+
+std::atomic<uint64_t> g_launches{0};
+thread_local char g_cuda_err[256] = "no error";
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ds_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return DS_ERR_CUDA;
+}
+
+// Call after each launch.
+ds_status launched() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DS_OK : cuda_fail(e);
+}
+
+ds_status check_dims(const ds_dims& d) {
+  if (d.B < 1 || d.Hq < 1 || d.Hkv < 1 || d.T_cap < 1 || d.r < 1 || d.d < 1)
+    return DS_ERR_INVALID_ARG;
+  if (d.Hq % d.Hkv != 0) return DS_ERR_INVALID_ARG;
+  if (d.r > d.d) return DS_ERR_INVALID_ARG;
+  if (d.d != kHeadDim) return DS_ERR_UNSUPPORTED;
+  // grid-dimension limits of the launches below
+  if ((int64_t)d.B * d.Hq > 65535 || (int64_t)d.B * d.Hkv > 65535) return DS_ERR_UNSUPPORTED;
+  return DS_OK;
+}
+
+// ---- split plan for the attention kernels (device independent) -------------
+// Heads are cut into S splits of rows_per_split rows so that the grid has
+// about kTargetCtas CTAs, no split is smaller than kMinRowsPerSplit rows
+// unless the head itself is, and sparse splits fit their index list in
+// shared memory.
+constexpr int kTargetCtas = 148 * 4;
+constexpr int kMinRowsPerSplit = 128;
+
+struct SplitPlan {
+  int S;
+  int rows_per_split;
+};
+
+SplitPlan plan_splits(int heads, int rows, bool sparse) {
+  int S = (kTargetCtas + heads - 1) / heads;
+  S = std::min(S, (rows + kMinRowsPerSplit - 1) / kMinRowsPerSplit);
+  if (sparse) S = std::max(S, (rows + kMaxRowsPerSplitSparse - 1) / kMaxRowsPerSplitSparse);
+  S = std::max(S, 1);
+  int rps = (rows + S - 1) / S;
+  rps = (rps + 3) & ~3;
+  S = (rows + rps - 1) / rps;
+  return {S, rps};
+}
+
+size_t partial_bytes(int heads, const SplitPlan& sp) {
+  if (sp.S <= 1) return 0;
+  size_t b = (size_t)heads * sp.S * kPartialStride * sizeof(float);
+  return (b + 255) & ~size_t(255);
+}
+
+size_t attend_smem(const SplitPlan& sp, bool sparse) {
+  size_t b = (size_t)kAttnWarps * kAttnStages * kAttnStageU4 * 16 + kAttnWarps * 132 * 4;
+  if (sparse) b += (size_t)sp.rows_per_split * 4;
+  return b;
+}
+
+// ---- per-device one-time kernel attributes ----------------------------------
+constexpr int kMaxDevices = 64;
+std::once_flag g_attr_once[kMaxDevices];
+cudaError_t g_attr_err[kMaxDevices];
+
+template <class Kern>
+cudaError_t allow_smem(Kern k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <class Src>
+cudaError_t topk_attrs() {
+  cudaError_t e = allow_smem(k_topk<Src>, TopkSmem::bytes(kMaxKeysPerCta));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_topk<Src>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
+ds_status ensure_attrs() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return DS_ERR_UNSUPPORTED;
+  std::call_once(g_attr_once[dev], [dev] {
+    cudaError_t r = cudaSuccess;
+    auto acc = [&r](cudaError_t x) {
+      if (r == cudaSuccess) r = x;
+    };
+    const size_t attn_max = (size_t)kAttnWarps * kAttnStages * kAttnStageU4 * 16 +
+                            kAttnWarps * 132 * 4 + (size_t)kMaxRowsPerSplitSparse * 4;
+    acc(allow_smem(k_attend<true>, attn_max));
+    acc(allow_smem(k_attend<false>, attn_max));
+    acc(topk_attrs<ScoresSource>());
+    acc(topk_attrs<LabelSource<8>>());
+    acc(topk_attrs<LabelSource<16>>());
+    acc(topk_attrs<LabelSource<32>>());
+    acc(topk_attrs<LabelSource<64>>());
+    acc(topk_attrs<LabelSource<128>>());
+    g_attr_err[dev] = r;
+  });
+  return g_attr_err[dev] == cudaSuccess ? DS_OK : cuda_fail(g_attr_err[dev]);
+}
+
+// ---- top-k launch -----------------------------------------------------------
+struct TopkPlan {
+  int cs;
+  int chunk;
+};
+
+bool plan_topk(int BH, int T, TopkPlan* out) {
+  int cs = (T + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
+  if (cs > kMaxCluster) return false;
+  // more CTAs per head when there are few heads, keeping >= 4096 keys per CTA
+  const int want = (2 * 148 + BH - 1) / BH;
+  cs = std::max(cs, std::min({want, kMaxCluster, std::max(1, T / 4096)}));
+  int chunk = (T + cs - 1) / cs;
+  chunk = (chunk + 31) & ~31;
+  cs = (T + chunk - 1) / chunk;
+  out->cs = cs;
+  out->chunk = chunk;
+  return true;
+}
+
+template <class Src>
+ds_status launch_topk(const Src& src, int32_t* idx, int BH, int T, int k, cudaStream_t st) {
+  TopkPlan tp;
+  if (!plan_topk(BH, T, &tp)) return DS_ERR_UNSUPPORTED;
+  const size_t smem = TopkSmem::bytes(tp.chunk);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tp.cs, BH, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = tp.cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = tp.cs > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_topk<Src>, src, idx, T, k, tp.chunk);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return launched();
+}
+
+ds_status launch_score(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
+                       const ds_dims& d, int T, cudaStream_t st) {
+  const int BH = d.B * d.Hq;
+  auto vec = [&](auto kern, int tokens_per_cta) {
+    dim3 grid((T + tokens_per_cta - 1) / tokens_per_cta, BH);
+    kern<<<grid, kScoreThreads, 0, st>>>(Q, C, label, scores, d.Hq, d.T_cap, T);
+    return launched();
+  };
+  switch (d.r) {
+    case 8: return vec(k_score_vec<8>, ScoreShape<8>::kTokensPerCta);
+    case 16: return vec(k_score_vec<16>, ScoreShape<16>::kTokensPerCta);
+    case 32: return vec(k_score_vec<32>, ScoreShape<32>::kTokensPerCta);
+    case 64: return vec(k_score_vec<64>, ScoreShape<64>::kTokensPerCta);
+    case 128: return vec(k_score_vec<128>, ScoreShape<128>::kTokensPerCta);
+    default: {
+      dim3 grid((T + kScoreThreads - 1) / kScoreThreads, BH);
+      k_score_any<<<grid, kScoreThreads, 0, st>>>(Q, C, label, scores, d.Hq, d.T_cap, T, d.r);
+      return launched();
+    }
+  }
+}
+
+template <int R>
+ds_status fused_topk(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
+                     int32_t* idx, const ds_dims& d, int T, int k, cudaStream_t st) {
+  LabelSource<R> src{Q, C, label, scores, d.Hq, d.T_cap};
+  return launch_topk(src, idx, d.B * d.Hq, T, k, st);
+}
+
+// Host-side checks of the split plan and workspace (no CUDA calls).
+ds_status check_attend_ws(const ds_dims& d, int rows, bool sparse, const void* ws,
+                          size_t ws_bytes) {
+  const int BH = d.B * d.Hq;
+  const SplitPlan sp = plan_splits(BH, rows, sparse);
+  const size_t need = partial_bytes(BH, sp);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return DS_ERR_WORKSPACE;
+  if (sp.S > 65535) return DS_ERR_UNSUPPORTED;
+  return DS_OK;
+}
+
+ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const void* V,
+                        const int32_t* idx, float* O, float* lse, int T, int rows, float scale,
+                        void* ws, cudaStream_t st) {
+  const bool sparse = idx != nullptr;
+  const int BH = d.B * d.Hq;
+  const SplitPlan sp = plan_splits(BH, rows, sparse);
+
+  AttnParams p;
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.idx = idx;
+  p.O = O;
+  p.lse = lse;
+  p.partial = static_cast<float*>(ws);
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.T_cap = d.T_cap;
+  p.T = T;
+  p.rows = rows;
+  p.rows_per_split = sp.rows_per_split;
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  dim3 grid(d.Hq / d.Hkv, sp.S, d.B * d.Hkv);
+  const size_t smem = attend_smem(sp, sparse);
+  if (sparse)
+    k_attend<true><<<grid, kAttnThreads, smem, st>>>(p);
+  else
+    k_attend<false><<<grid, kAttnThreads, smem, st>>>(p);
+  ds_status s = launched();
+  if (s != DS_OK || sp.S == 1) return s;
+  k_lse_merge<<<BH, kHeadDim, 0, st>>>(p.partial, O, lse, sp.S);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ds_status_string(ds_status s) {
+  switch (s) {
+    case DS_OK: return "DS_OK";
+    case DS_ERR_INVALID_ARG: return "DS_ERR_INVALID_ARG";
+    case DS_ERR_UNSUPPORTED: return "DS_ERR_UNSUPPORTED";
+    case DS_ERR_WORKSPACE: return "DS_ERR_WORKSPACE";
+    case DS_ERR_CUDA: return "DS_ERR_CUDA";
+  }
+  return "DS_ERR_UNKNOWN";
+}
+
+const char* ds_last_cuda_error(void) { return g_cuda_err; }
+
+uint64_t ds_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
+  if (check_dims(dims) != DS_OK || T < 1 || T > dims.T_cap) return 0;
+  const int BH = dims.B * dims.Hq;
+  switch (op) {
+    case DS_OP_SPARSE_DECODE:
+      if (k < 1 || k > T) return 0;
+      return partial_bytes(BH, plan_splits(BH, k, true));
+    case DS_OP_DECODE:
+      return partial_bytes(BH, plan_splits(BH, T, false));
+    default:
+      return 0;
+  }
+}
+
+ds_status ds_device_status(uint32_t* bits, int32_t clear, ds_stream_t stream) {
+  if (!bits) return DS_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_status, &z, sizeof(z));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *bits = v;
+  return DS_OK;
+}
+
+ds_status ds_label_append(const void* K, const int32_t* C, void* label, ds_dims dims, int32_t t0,
+                          int32_t n, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!K || !C || !label || !aligned16(K) || !aligned16(C) || !aligned16(label))
+    return DS_ERR_INVALID_ARG;
+  if (t0 < 0 || n < 1 || (int64_t)t0 + n > dims.T_cap) return DS_ERR_INVALID_ARG;
+  const int G = dims.Hq / dims.Hkv;
+  const size_t cs_bytes = (size_t)G * dims.r * sizeof(int32_t);
+  if (cs_bytes > 40 * 1024) return DS_ERR_UNSUPPORTED;
+  dim3 grid((n + kLabelTile - 1) / kLabelTile, dims.B * dims.Hkv);
+  k_label_append<<<grid, kLabelThreads, cs_bytes, stream>>>(
+      static_cast<const uint16_t*>(K), C, static_cast<uint16_t*>(label), dims.Hq, dims.Hkv,
+      dims.T_cap, dims.r, t0, n);
+  return launched();
+}
+
+ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* scores,
+                   ds_dims dims, int32_t T, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !C || !label || !scores || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
+      !aligned16(scores))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
+  return launch_score(static_cast<const uint16_t*>(Q), C, static_cast<const uint16_t*>(label),
+                      scores, dims, T, stream);
+}
+
+ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int32_t k, void* ws,
+                  size_t ws_bytes, ds_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!scores || !idx || !aligned16(scores) || !aligned16(idx)) return DS_ERR_INVALID_ARG;
+  if (BH < 1 || T < 1 || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (BH > 65535 || T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
+  ds_status s = ensure_attrs();
+  if (s != DS_OK) return s;
+  return launch_topk(ScoresSource{scores}, idx, BH, T, k, stream);
+}
+
+ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
+                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !C || !label || !idx || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
+      !aligned16(idx) || (scores && !aligned16(scores)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
+  const bool fused = dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 || dims.r == 128;
+  if (!fused && !scores) return DS_ERR_UNSUPPORTED;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  auto Qb = static_cast<const uint16_t*>(Q);
+  auto Lb = static_cast<const uint16_t*>(label);
+  switch (dims.r) {
+    case 8: return fused_topk<8>(Qb, C, Lb, scores, idx, dims, T, k, stream);
+    case 16: return fused_topk<16>(Qb, C, Lb, scores, idx, dims, T, k, stream);
+    case 32: return fused_topk<32>(Qb, C, Lb, scores, idx, dims, T, k, stream);
+    case 64: return fused_topk<64>(Qb, C, Lb, scores, idx, dims, T, k, stream);
+    case 128: return fused_topk<128>(Qb, C, Lb, scores, idx, dims, T, k, stream);
+    default:
+      // other r: two launches through the caller's score buffer
+      s = launch_score(Qb, C, Lb, scores, dims, T, stream);
+      if (s != DS_OK) return s;
+      return launch_topk(ScoresSource{scores}, idx, dims.B * dims.Hq, T, k, stream);
+  }
+}
+
+ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
+                           float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
+                           void* ws, size_t ws_bytes, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  s = check_attend_ws(dims, k, true, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
+}
+
+ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float* lse,
+                    ds_dims dims, int32_t T, float scale, void* ws, size_t ws_bytes,
+                    ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
+  s = check_attend_ws(dims, T, false, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  return launch_attend(dims, Q, K, V, nullptr, O, lse, T, T, scale, ws, stream);
+}
+
+}  // extern "C"

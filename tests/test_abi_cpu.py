@@ -1,0 +1,161 @@
+"""The C ABI on a machine without a GPU: symbols, host-side validation, sizes.
+
+Nothing here launches a kernel: every call below is rejected by the host-side
+argument checks before the library touches the CUDA runtime.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+import post_token_sparse_b200 as ds
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ds.h")
+FAKE = 0x7000_0000_0000  # aligned, never dereferenced: the calls fail validation first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ds_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for want in ("ds_label_append", "ds_score", "ds_topk", "ds_score_topk", "ds_sparse_decode",
+                 "ds_decode", "ds_workspace_size", "ds_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ds.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", ds.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (ds_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings():
+    lib = ds.lib()
+    assert lib.ds_status_string(0) == b"DS_OK"
+    assert lib.ds_status_string(1) == b"DS_ERR_INVALID_ARG"
+    assert lib.ds_status_string(2) == b"DS_ERR_UNSUPPORTED"
+    assert lib.ds_status_string(3) == b"DS_ERR_WORKSPACE"
+    assert lib.ds_status_string(4) == b"DS_ERR_CUDA"
+
+
+def _dims(**kw):
+    base = dict(B=2, Hq=8, Hkv=2, d=128, T_cap=1000, r=16)
+    base.update(kw)
+    return ds.Dims(base["B"], base["Hq"], base["Hkv"], base["d"], base["T_cap"], base["r"])
+
+
+P = ctypes.c_void_p(FAKE)
+NUL = None
+
+
+@pytest.mark.parametrize("dims,want", [
+    (dict(B=0), ds.DS_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), ds.DS_ERR_INVALID_ARG),
+    (dict(r=0), ds.DS_ERR_INVALID_ARG),
+    (dict(r=129), ds.DS_ERR_INVALID_ARG),
+    (dict(d=64, r=8), ds.DS_ERR_UNSUPPORTED),
+    (dict(B=70000), ds.DS_ERR_UNSUPPORTED),
+])
+def test_bad_dims(dims, want):
+    lib = ds.lib()
+    d = _dims(**dims)
+    assert lib.ds_label_append(P, P, P, d, 0, 1, NUL) == want
+    assert lib.ds_score(P, P, P, P, d, 10, NUL) == want
+    assert lib.ds_score_topk(P, P, P, NUL, P, d, 10, 5, NUL) == want
+    assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0, NUL) == want
+    assert lib.ds_decode(P, P, P, P, NUL, d, 10, 1.0, NUL, 0, NUL) == want
+
+
+def test_bad_sizes_and_pointers():
+    lib = ds.lib()
+    d = _dims()
+    bad = ds.DS_ERR_INVALID_ARG
+    mis = ctypes.c_void_p(FAKE + 4)
+    # label append range
+    assert lib.ds_label_append(P, P, P, d, -1, 1, NUL) == bad
+    assert lib.ds_label_append(P, P, P, d, 0, 0, NUL) == bad
+    assert lib.ds_label_append(P, P, P, d, 990, 11, NUL) == bad
+    assert lib.ds_label_append(NUL, P, P, d, 0, 1, NUL) == bad
+    assert lib.ds_label_append(mis, P, P, d, 0, 1, NUL) == bad
+    # score: T out of range, null/misaligned
+    assert lib.ds_score(P, P, P, P, d, 0, NUL) == bad
+    assert lib.ds_score(P, P, P, P, d, 1001, NUL) == bad
+    assert lib.ds_score(P, P, P, mis, d, 10, NUL) == bad
+    # top-k: k out of range
+    assert lib.ds_topk(P, P, 4, 10, 0, NUL, 0, NUL) == bad
+    assert lib.ds_topk(P, P, 4, 10, 11, NUL, 0, NUL) == bad
+    assert lib.ds_topk(P, P, 0, 10, 1, NUL, 0, NUL) == bad
+    assert lib.ds_topk(NUL, P, 4, 10, 1, NUL, 0, NUL) == bad
+    assert lib.ds_topk(P, mis, 4, 10, 1, NUL, 0, NUL) == bad
+    assert lib.ds_topk(P, P, 4, 16 * 40960 + 1, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_topk(P, P, 70000, 10, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
+    # fused score+topk: r not a multiple of 8 needs a score buffer
+    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 20, NUL) == bad
+    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 5, NUL) == ds.DS_ERR_UNSUPPORTED
+    # sparse decode: k > T, T > T_cap, misaligned lse
+    assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 10, 11, 1.0, NUL, 0, NUL) == bad
+    assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 1001, 5, 1.0, NUL, 0, NUL) == bad
+    assert lib.ds_sparse_decode(P, P, P, P, P, mis, d, 10, 5, 1.0, NUL, 0, NUL) == bad
+    assert lib.ds_decode(P, P, P, P, NUL, d, 0, 1.0, NUL, 0, NUL) == bad
+
+
+def test_workspace_checked_before_launch():
+    lib = ds.lib()
+    d = _dims(B=1, Hq=4, Hkv=4, T_cap=100000)
+    need = lib.ds_workspace_size(ds.OP_DECODE, d, 100000, 100000)
+    assert need > 0  # few heads, long rows: the rows are split
+    assert lib.ds_decode(P, P, P, P, NUL, d, 100000, 1.0, NUL, 0, NUL) == ds.DS_ERR_WORKSPACE
+    assert lib.ds_decode(P, P, P, P, NUL, d, 100000, 1.0, P, need - 1, NUL) == \
+        ds.DS_ERR_WORKSPACE
+    need_s = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 100000, 20000)
+    assert need_s > 0
+    assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 100000, 20000, 1.0, NUL, 0, NUL) == \
+        ds.DS_ERR_WORKSPACE
+
+
+def test_workspace_sizes():
+    lib = ds.lib()
+    # many heads, short rows: no split, no workspace
+    d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 512) == 0
+    assert lib.ds_workspace_size(ds.OP_TOPK, d, 32768, 512) == 0
+    assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == 0
+    # long single sequence: split, 132 floats per split, 256-byte rounded
+    d = _dims(B=1, Hq=32, Hkv=32, T_cap=262144, r=8)
+    n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 262144, 16384)
+    assert n > 0 and n % 256 == 0 and (n // (32 * 132 * 4)) >= 2
+    # invalid sizes give 0
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 0, 1) == 0
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 100, 101) == 0
+    assert lib.ds_workspace_size(ds.OP_DECODE, _dims(d=64), 100, 100) == 0
+    # depends only on the arguments
+    assert lib.ds_workspace_size(ds.OP_DECODE, d, 262144, 1) == \
+        lib.ds_workspace_size(ds.OP_DECODE, d, 262144, 1)
+
+
+def test_launch_counter_starts_untouched():
+    assert ds.kernel_launches() >= 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package with no libds.so must refuse to import."""
+    pkg = tmp_path / "post_token_sparse_b200"
+    pkg.mkdir()
+    src = open(os.path.join(os.path.dirname(ds.__file__), "__init__.py")).read()
+    (pkg / "__init__.py").write_text(src)
+    res = subprocess.run([sys.executable, "-c", "import post_token_sparse_b200"],
+                         cwd=tmp_path, capture_output=True, text=True)
+    assert res.returncode != 0
+    assert "libds.so is missing" in res.stderr
