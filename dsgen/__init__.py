@@ -17,7 +17,7 @@ import threading
 
 import numpy as np
 
-from .configs import CONFIGS, Workload, workload  # noqa: F401
+from .configs import CONFIGS, ORDER, Workload, workload  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gen.c")
