@@ -174,6 +174,40 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
                     ds_stream_t stream);
 
 /*
+ * ds_sparse_decode_noalloc -- ds_sparse_decode for callers that cannot
+ * allocate device memory.  (The paper has no counterpart: this is a property
+ * of the library's interface, not of the method.)
+ *
+ * Some callers cannot hand the library a workspace: a serving loop that
+ * reserved all of HBM for its KV cache at start-up and forbids further
+ * allocation (so a request can never fail with out-of-memory half-way), code
+ * on a latency-critical path where cudaMalloc's implicit device-wide
+ * synchronisation is unacceptable, or a plug-in that is given only its input
+ * and output buffers by a host framework that owns all device memory.  This
+ * call computes exactly what ds_sparse_decode computes, with the same kernels
+ * and the same split plan, but keeps the split partials in a fixed array
+ * inside the library (DS_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU
+ * that loads the library until the process exits).  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Arguments as for ds_sparse_decode, without ws / ws_bytes.  Returns
+ * DS_ERR_WORKSPACE, launching nothing, when the partials these sizes need
+ * (ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k)) exceed
+ * DS_NOALLOC_SCRATCH_BYTES.
+ *
+ * The first call on each device looks up the array's device address with
+ * that device current (cudaGetSymbolAddress); make that first call outside
+ * any stream capture.  All calls on a device share the one array and it keeps
+ * the previous call's contents (nothing in it needs to start at zero): calls
+ * that may overlap on the GPU -- on different streams without an ordering
+ * between them -- race on it and must not be issued.
+ */
+#define DS_NOALLOC_SCRATCH_BYTES (4u << 20)
+ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,
+                                   const int32_t* idx, float* O, float* lse, ds_dims dims,
+                                   int32_t T, int32_t k, float scale, ds_stream_t stream);
+
+/*
  * Bytes of device workspace `op` needs for these sizes (0 if none).  Depends
  * only on the arguments, never on the device.  Returns 0 for invalid sizes.
  */

@@ -213,3 +213,26 @@ def device_status(clear: bool = True, device=None) -> int:
 def kernel_launches() -> int:
     """Kernels launched by libds.so in this process so far."""
     return int(_lib.ds_kernel_launches())
+
+
+# ---------------------------------------------------------------------------
+# sparse decode for callers that cannot allocate device memory
+
+_lib.ds_sparse_decode_noalloc.argtypes = [ctypes.c_void_p] * 6 + [
+    Dims, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p]
+_lib.ds_sparse_decode_noalloc.restype = ctypes.c_int
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def sparse_decode_noalloc(Q, K, V, idx, O, T: int, scale: float, lse=None):
+    """sparse_decode without a workspace: the split partials use a fixed array
+    inside the library (NOALLOC_SCRATCH_BYTES per GPU).  For callers that must not
+    allocate device memory on their decode path; see ds_sparse_decode_noalloc in
+    include/ds.h for the sharing rule (calls that overlap on the GPU race)."""
+    dims = dims_of(Q, K, 1)
+    k = idx.shape[-1]
+    _check(_lib.ds_sparse_decode_noalloc(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
+        _ptr(idx, torch.int32, "idx"), _ptr(O, torch.float32, "O"),
+        _ptr(lse, torch.float32, "lse"), dims, T, k, scale, _stream(Q.device)),
+        "ds_sparse_decode_noalloc")

@@ -398,3 +398,56 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
 }
 
 }  // extern "C"
+
+// ---- sparse decode with library-owned scratch ---------------------------------
+// For callers that must not allocate device memory: the split partials live in
+// this fixed file-scope array instead of a caller workspace.  Every call on a
+// device shares it, so calls that overlap on the GPU race on it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::once_flag g_scratch_once[kMaxDevices];
+void* g_scratch_addr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side handle, so the address is looked up once
+// per device, with that device current.
+ds_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return DS_ERR_UNSUPPORTED;
+  std::call_once(g_scratch_once[dev], [dev] {
+    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_noalloc_scratch);
+  });
+  if (g_scratch_err[dev] != cudaSuccess) return cuda_fail(g_scratch_err[dev]);
+  *out = g_scratch_addr[dev];
+  return DS_OK;
+}
+}  // namespace
+
+extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,
+                                              const int32_t* idx, float* O, float* lse,
+                                              ds_dims dims, int32_t T, int32_t k, float scale,
+                                              ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  const int BH = dims.B * dims.Hq;
+  const SplitPlan sp = plan_splits(BH, k, true);
+  const size_t need = partial_bytes(BH, sp);
+  if (need > DS_NOALLOC_SCRATCH_BYTES) return DS_ERR_WORKSPACE;
+  if (sp.S > 65535) return DS_ERR_UNSUPPORTED;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  void* scratch = nullptr;
+  if (need > 0) {
+    s = noalloc_scratch(&scratch);
+    if (s != DS_OK) return s;
+  }
+  return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
+}
