@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--unfused", action="store_true",
                    help="separate score and top-k launches instead of the fused one")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--batch", type=int, default=None,
+                   help="override the workload's batch size (smaller captures for ncu)")
     return p.parse_args()
 
 
@@ -481,6 +483,8 @@ def main():
     hbm_peak, peak_kind = peaks()
 
     base = dsgen.workload(args.workload)
+    if args.batch:
+        base = base.with_(B=args.batch)
     w = base.with_(seed=base.seed + rank)  # independent replica per rank
     step = Step(w, fused=not args.unfused)
 

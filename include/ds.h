@@ -125,7 +125,7 @@ ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* sc
  * the contract (no fault, unspecified choice).  Token selection by the higher
  * activation (Double Sparsity page, Method details: Key design).
  *
- * Requires 1 <= k <= T <= 655360 and BH <= 65535.  Needs no workspace
+ * Requires 1 <= k <= T <= 1048576 and BH <= 65535.  Needs no workspace
  * (ds_workspace_size returns 0); `ws` may be NULL.
  */
 ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int32_t k,

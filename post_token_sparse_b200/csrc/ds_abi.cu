@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
@@ -99,7 +100,7 @@ cudaError_t allow_smem(Kern k, size_t bytes) {
 
 template <class Src>
 cudaError_t topk_attrs() {
-  cudaError_t e = allow_smem(k_topk<Src>, TopkSmem::bytes(kMaxKeysPerCta));
+  cudaError_t e = allow_smem(k_topk<Src>, TopkLayout(kMaxKeysPerCta, kMaxCluster).bytes());
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(k_topk<Src>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
@@ -135,12 +136,26 @@ struct TopkPlan {
   int chunk;
 };
 
-bool plan_topk(int BH, int T, TopkPlan* out) {
+// A head of at most kSample tokens is one CTA (it computes every key of the
+// head anyway).  Longer heads are cut so that one CTA's expected number of
+// candidates -- the tokens inside the sample bracket -- stays near half its
+// list, and, with few heads, further (down to kTopkMinKeys tokens per CTA) to
+// give every SM four CTAs.
+constexpr int kTopkMinKeys = 2048;
+
+bool plan_topk(int BH, int T, int k, TopkPlan* out) {
   int cs = (T + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
   if (cs > kMaxCluster) return false;
-  // more CTAs per head when there are few heads, keeping >= 4096 keys per CTA
-  const int want = (2 * 148 + BH - 1) / BH;
-  cs = std::max(cs, std::min({want, kMaxCluster, std::max(1, T / 4096)}));
+  if (T > kSample) {
+    const double p = (double)k / T, e = p * kSample;
+    const double frac = 2.0 * (kBracketSigmas * std::sqrt(e * (1.0 - p)) + 3.0) / kSample;
+    const double max_chunk = 0.5 * kCandCap / std::max(frac, 1e-9);
+    cs = std::max(cs, (int)std::min<double>(kMaxCluster, std::ceil(T / max_chunk)));
+    if (BH * cs < 4 * 148) {
+      const int want = (4 * 148 + BH - 1) / BH;
+      cs = std::max(cs, std::min({want, kMaxCluster, std::max(1, T / kTopkMinKeys)}));
+    }
+  }
   int chunk = (T + cs - 1) / cs;
   chunk = (chunk + 31) & ~31;
   cs = (T + chunk - 1) / chunk;
@@ -152,8 +167,8 @@ bool plan_topk(int BH, int T, TopkPlan* out) {
 template <class Src>
 ds_status launch_topk(const Src& src, int32_t* idx, int BH, int T, int k, cudaStream_t st) {
   TopkPlan tp;
-  if (!plan_topk(BH, T, &tp)) return DS_ERR_UNSUPPORTED;
-  const size_t smem = TopkSmem::bytes(tp.chunk);
+  if (!plan_topk(BH, T, k, &tp)) return DS_ERR_UNSUPPORTED;
+  const size_t smem = TopkLayout(tp.chunk, tp.cs).bytes();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tp.cs, BH, 1);
   cfg.blockDim = dim3(kTopkThreads, 1, 1);

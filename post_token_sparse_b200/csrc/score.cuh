@@ -16,9 +16,10 @@ constexpr int kScoreThreads = 256;
 // 16-byte chunks of one label row, and rows per thread per pass
 template <int R>
 struct ScoreShape {
-  static constexpr int kChunks = R / 8;                         // uint4 per row
-  static constexpr int kRowsPerThread = kChunks >= 4 ? 1 : 4 / kChunks;
-  static constexpr int kTokensPerCta = kScoreThreads * kRowsPerThread;
+  static constexpr int kLanes = R / 8;                 // lanes (16-byte chunks) per row
+  static constexpr int kRowsPerInstr = 32 / kLanes;    // rows per warp load
+  static constexpr int kSlots = 4;                     // loads in flight per thread
+  static constexpr int kTokensPerCta = (kScoreThreads / 32) * kSlots * kRowsPerInstr;
 };
 
 // fp32 q[C] for one head into shared memory (channel ids masked into range)
@@ -35,28 +36,47 @@ __device__ __forceinline__ void load_qc(const uint16_t* __restrict__ Q,
   }
 }
 
-// Score of one label row whose chunks are already in registers.  Summation is
-// sequential over j so the result does not depend on R's blocking.
-template <int R>
-__device__ __forceinline__ float row_score(const uint4 (&v)[R / 8], const float* qs) {
-  float a = 0.f;
-#pragma unroll
-  for (int c = 0; c < R / 8; ++c) {
-    const uint4 x = v[c];
-    const float* q = qs + 8 * c;
-    a = fmaf(bf_lo(x.x), q[0], a);
-    a = fmaf(bf_hi(x.x), q[1], a);
-    a = fmaf(bf_lo(x.y), q[2], a);
-    a = fmaf(bf_hi(x.y), q[3], a);
-    a = fmaf(bf_lo(x.z), q[4], a);
-    a = fmaf(bf_hi(x.z), q[5], a);
-    a = fmaf(bf_lo(x.w), q[6], a);
-    a = fmaf(bf_hi(x.w), q[7], a);
-  }
+// Scores are summed in a fixed order shared by every kernel that computes
+// them, so the fused score+select path and this one give identical fp32
+// values: each 16-byte chunk (8 channels) is summed sequentially, then the
+// r/8 chunk sums are added pairwise ((c0+c1)+(c2+c3))+... -- the order a
+// butterfly of xor-shuffles produces when r/8 lanes share a row.
+__device__ __forceinline__ float chunk_dot(const uint4& x, const float* q) {
+  float a = bf_lo(x.x) * q[0];
+  a = fmaf(bf_hi(x.x), q[1], a);
+  a = fmaf(bf_lo(x.y), q[2], a);
+  a = fmaf(bf_hi(x.y), q[3], a);
+  a = fmaf(bf_lo(x.z), q[4], a);
+  a = fmaf(bf_hi(x.z), q[5], a);
+  a = fmaf(bf_lo(x.w), q[6], a);
+  a = fmaf(bf_hi(x.w), q[7], a);
   return a;
 }
 
-// grid: (ceil(T / kTokensPerCta), B*Hq).  R is a multiple of 8 (rows are whole uint4s).
+// One thread, whole row in registers (the same tree as the lane butterfly).
+template <int R>
+__device__ __forceinline__ float row_score(const uint4 (&v)[R / 8], const float* qs) {
+  float part[R / 8];
+#pragma unroll
+  for (int c = 0; c < R / 8; ++c) part[c] = chunk_dot(v[c], qs + 8 * c);
+#pragma unroll
+  for (int st = 1; st < R / 8; st <<= 1)
+#pragma unroll
+    for (int c = 0; c < R / 8; c += 2 * st) part[c] = part[c] + part[c + st];
+  return part[0];
+}
+
+// r/8 consecutive lanes hold the chunks of one row: butterfly sum of the chunk dots.
+template <int R>
+__device__ __forceinline__ float lane_group_score(const uint4& x, const float* qs, int chunk) {
+  float a = chunk_dot(x, qs + 8 * chunk);
+#pragma unroll
+  for (int st = 1; st < R / 8; st <<= 1) a = a + __shfl_xor_sync(0xffffffffu, a, st);
+  return a;
+}
+
+// grid: (ceil(T / kTokensPerCta), B*Hq).  R is a multiple of 8 (rows are whole
+// uint4s).  r/8 lanes share a row, so every warp load reads 512 contiguous bytes.
 template <int R>
 __global__ void __launch_bounds__(kScoreThreads)
 k_score_vec(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
@@ -70,21 +90,24 @@ k_score_vec(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
 
   const uint4* lab = reinterpret_cast<const uint4*>(label + (size_t)bh * T_cap * R);
   float* out = scores + (size_t)bh * T;
-  const int tbase = blockIdx.x * S::kTokensPerCta + threadIdx.x;
-
-  uint4 v[S::kRowsPerThread][S::kChunks];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = lane % S::kLanes;
+  // token of slot i of this lane
+  auto token = [&](int i) {
+    return blockIdx.x * S::kTokensPerCta + (warp * S::kSlots + i) * S::kRowsPerInstr +
+           lane / S::kLanes;
+  };
+  uint4 v[S::kSlots];
 #pragma unroll
-  for (int i = 0; i < S::kRowsPerThread; ++i) {
-    const int t = tbase + i * kScoreThreads;
-    if (t < T) {
-#pragma unroll
-      for (int c = 0; c < S::kChunks; ++c) v[i][c] = ldg_stream(lab + (size_t)t * S::kChunks + c);
-    }
+  for (int i = 0; i < S::kSlots; ++i) {
+    const int t = token(i);
+    if (t < T) v[i] = ldg_stream(lab + (size_t)t * S::kLanes + chunk);
   }
 #pragma unroll
-  for (int i = 0; i < S::kRowsPerThread; ++i) {
-    const int t = tbase + i * kScoreThreads;
-    if (t < T) out[t] = row_score<R>(v[i], qs);
+  for (int i = 0; i < S::kSlots; ++i) {
+    const int t = token(i);
+    const float s = lane_group_score<R>(v[i], qs, chunk);  // all lanes take part
+    if (t < T && chunk == 0) out[t] = s;
   }
 }
 

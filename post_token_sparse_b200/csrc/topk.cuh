@@ -1,28 +1,41 @@
-// Per-head top-k by radix select over shared-memory-resident keys.
+// Per-head top-k: sample-bracketed selection in one streaming pass.
 //
 // Token selection keeps the tokens with the highest approximate activation
 // (Double Sparsity, Method details: Key design).  Contract: the k largest
 // scores, ties to the lower token index, -0 == +0, output ascending.
 //
-// One thread-block cluster per head (cluster size CS = 1..16).  CTA c of the
-// cluster owns the contiguous token range [c*chunk, min((c+1)*chunk, T)) and
-// keeps its order-preserving uint32 keys in shared memory for the whole
-// selection, so scores are read (or computed from the label cache) once.
+// One thread-block cluster per head (cluster size CS = 1..16); CTA c owns the
+// tokens [c*chunk, min((c+1)*chunk, T)).  No CTA stores its keys: shared
+// memory holds two bit masks and a short candidate list, so four CTAs share
+// an SM and one CTA's selection work overlaps the others' streaming.
 //
-//   1. fill    keys + local histogram of digit 0 (key bits 31..21)
-//   2. digit   local histograms are added into CTA 0's shared memory through
-//              distributed shared memory; after a cluster barrier every CTA
-//              reads the merged histogram and finds the bin holding the k-th
-//              largest key.  Digits: bits 31..21, 20..10, 9..0.  If the bin's
-//              whole population is needed, selection is "key >= bin start"
-//              and the remaining digits are skipped.
-//   3. output  two passes over the keys: per-warp counts of (key > thr) and
-//              (key == thr), a cluster-wide exclusive scan of the per-CTA
-//              counts (read through distributed shared memory), then warp
-//              ballots place each selected index at its rank: ascending
-//              order and the lower-index tie rule fall out of the scan order.
+//   1. sample   exact keys of a stratified sample of the whole head: 128
+//               blocks of 32 consecutive tokens spread over [0, T), or every
+//               token when T <= 4096.  Every CTA of a cluster draws the same
+//               sample, so all of them agree on what follows without talking.
+//   2. bracket  radix select on the sample: with the whole head sampled, the
+//               exact k-th key (lo = hi = threshold); otherwise the sample's
+//               keys at ranks k*m/T -/+ (5 standard deviations + 2) become
+//               hi / lo: keys above hi are selected, keys below lo are not.
+//   3. stream   one pass over this CTA's keys (computed from the label cache,
+//               or read from the scores): key > hi sets a bit of the "above"
+//               mask; lo <= key <= hi sets a bit of the "equal" mask when
+//               lo == hi, else goes to the candidate list (exact key, token).
+//   4. check    cluster totals must put the k-th key inside [lo, hi] with no
+//               list overflow.  If not (a sample miss, or heavy ties), exact
+//               refinement takes over: one histogram pass per key digit
+//               narrows the bracket to the bin holding the k-th key and the
+//               stream pass repeats; a one-value bracket always fits.
+//   5. resolve  radix select of the remaining rank over the candidate lists
+//               (histograms merged over the cluster) gives the exact threshold
+//               key; candidates above it join the "above" mask, candidates
+//               equal to it the "equal" mask.
+//   6. write    per-warp counts, a cluster-wide exclusive scan (pushed into the
+//               later CTAs before a barrier), then one 32-token group per lane:
+//               indices in ascending order, ties taken in index order.
 //
-// Synchronisation is by hardware cluster / CTA barriers only; no spin waits.
+// Synchronisation is by hardware CTA / cluster barriers only; no spin waits.
+// No CTA touches another's shared memory after the last cluster barrier.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -34,30 +47,52 @@ namespace ds {
 
 namespace cg = cooperative_groups;
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kMaxCluster = 16;
-constexpr int kMaxKeysPerCta = 40960;
+constexpr int kMaxKeysPerCta = 65536;
+constexpr int kSample = 4096;                // sample size (the whole head when T <= kSample)
+constexpr int kSampleBlocks = kSample / 32;  // 128 blocks of 32 consecutive tokens
+constexpr int kCandCap = 4096;               // candidate list of one CTA
+constexpr float kBracketSigmas = 5.f;
+
 // digits of the 32-bit key: bits 31..21, 20..10, 9..0
 __host__ __device__ constexpr int digit_shift(int d) { return d == 0 ? 21 : (d == 1 ? 10 : 0); }
 __host__ __device__ constexpr int digit_bits(int d) { return d == 2 ? 10 : 11; }
 __host__ __device__ constexpr int digit_bins(int d) { return 1 << digit_bits(d); }
-constexpr int kBinsPerThread = 2048 / kTopkThreads;  // 4
+constexpr int kBinsPerThread = 2048 / kTopkThreads;  // 8
 
-// Shared-memory layout (32-bit words); keys follow.
-struct TopkSmem {
-  static constexpr int kHist = 0;                   // local histogram [2048]
-  static constexpr int kMerged0 = kHist + 2048;     // merged digit 0 (used in CTA 0)
-  static constexpr int kMerged1 = kMerged0 + 2048;  // merged digit 1
-  static constexpr int kMerged2 = kMerged1 + 2048;  // merged digit 2 [1024]; kMerged0 + 2048*d
-  static constexpr int kWarpGt = kMerged2 + 1024;   // per-warp counts
-  static constexpr int kWarpEq = kWarpGt + kTopkWarps;
-  static constexpr int kScan = kWarpEq + kTopkWarps;  // block-scan scratch [kTopkWarps]
-  static constexpr int kMisc = kScan + kTopkWarps;    // 16 words of broadcast values
-  static constexpr int kKeys = kMisc + 16;
-  static constexpr size_t bytes(int keys) { return (size_t)(kKeys + keys) * 4; }
+// Shared-memory layout in 32-bit words (depends on the chunk and cluster size).
+struct TopkLayout {
+  int merged0, merged1, small, masks, X, words;
+  __host__ __device__ TopkLayout(int chunk, int cs) {
+    int o = 2048;  // histogram (2048 bins) at 0
+    merged0 = o;   // cluster-merged histograms (CTA-local copies)
+    if (cs > 1) o += 2048;
+    merged1 = o;
+    if (cs > 1) o += 2048;
+    small = o;  // misc[32], warp_gt[8], warp_eq[8], scan[16], q[C] as fp32 [128]
+    o += 192;
+    masks = o;  // per 32-token group: "above" bits, then "equal" bits
+    o += 2 * (chunk / 32);
+    o = (o + 3) & ~3;
+    X = o;  // candidates: keys [kCandCap], tokens [kCandCap]; while sampling, the
+            // sample keys in the first half and two histograms in the second
+    o += 2 * kCandCap;
+    words = o;
+  }
+  __host__ __device__ size_t bytes() const { return (size_t)words * 4; }
 };
-enum { M_BIN = 0, M_ABOVE = 1, M_CNT = 2, M_CTA_GT = 3, M_CTA_EQ = 4 };
+static_assert(kSample <= kCandCap, "sample keys live in the candidate-key half");
+static_assert(2 * 2048 <= kCandCap, "two sample histograms live in the token half");
+
+enum {
+  M_BIN = 0, M_ABOVE = 1, M_CNT = 2,     // find_bins, target 1
+  M_BIN2 = 3, M_ABOVE2 = 4, M_CNT2 = 5,  // find_bins, target 2
+  M_NCAND = 6,                           // this CTA's candidate count
+  M_TOT = 8,                             // cluster totals: above, equal, cand, overflow
+  M_GT_BEFORE = 12, M_EQ_BEFORE = 13     // counts of the earlier CTAs of the cluster
+};
 
 __device__ __forceinline__ void cluster_or_cta_sync(int cs) {
   if (cs > 1)
@@ -83,11 +118,11 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   return wbase + incl - v;
 }
 
-// Finds the bin b (counting bins from the top) such that
-// count(bins > b) < krem <= count(bins >= b) and writes b, count(bins > b)
-// and count(b) to misc.  `hist` may point into another CTA's shared memory.
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t krem,
-                                         uint32_t* scratch, uint32_t* misc) {
+// For rank r (1 = largest) finds the bin b (bins counted from the top) with
+// count(bins > b) < r <= count(bins >= b) and writes b, count(bins > b) and
+// count(b) to out[0..2]; r == 0 finds nothing.
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t r,
+                                         uint32_t* scratch, uint32_t* out) {
   uint32_t c[kBinsPerThread];
   uint32_t sum = 0;
 #pragma unroll
@@ -97,14 +132,14 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32
     sum += c[j];
   }
   const uint32_t above = block_exclusive_scan(sum, scratch);
-  if (sum > 0 && above < krem && krem <= above + sum) {
+  if (r && sum > 0 && above < r && r <= above + sum) {
     uint32_t acc = above;
 #pragma unroll
     for (int j = 0; j < kBinsPerThread; ++j) {
-      if (acc + c[j] >= krem) {
-        misc[M_BIN] = (uint32_t)(nbins - 1 - (threadIdx.x * kBinsPerThread + j));
-        misc[M_ABOVE] = acc;
-        misc[M_CNT] = c[j];
+      if (acc + c[j] >= r) {
+        out[0] = (uint32_t)(nbins - 1 - (threadIdx.x * kBinsPerThread + j));
+        out[1] = acc;
+        out[2] = c[j];
         break;
       }
       acc += c[j];
@@ -113,208 +148,493 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32
   __syncthreads();
 }
 
+// hist (nbins bins) summed over the cluster into every CTA's merged copy;
+// returns the histogram to read (the local one when cs == 1).
+__device__ __forceinline__ const uint32_t* cluster_hist(uint32_t* hist, uint32_t* merged,
+                                                        int nbins, int cs) {
+  if (cs == 1) return hist;
+  cg::cluster_group cl = cg::this_cluster();
+  for (int i = threadIdx.x; i < nbins; i += kTopkThreads) {
+    const uint32_t v = hist[i];
+    if (v)
+      for (int c = 0; c < cs; ++c) atomicAdd(cl.map_shared_rank(merged, c) + i, v);
+  }
+  cl.sync();
+  return merged;
+}
+
+// Four counters summed over the cluster into misc[M_TOT..M_TOT+3] of every CTA
+// (those words must be zero everywhere; the caller zeroes them after use,
+// before its next cluster barrier).
+__device__ __forceinline__ void cluster_totals(uint32_t* misc, const uint32_t (&v)[4], int cs) {
+  if (threadIdx.x == 0) {
+    if (cs == 1) {
+      for (int i = 0; i < 4; ++i) misc[M_TOT + i] = v[i];
+    } else {
+      cg::cluster_group cl = cg::this_cluster();
+      for (int c = 0; c < cs; ++c) {
+        uint32_t* m = cl.map_shared_rank(misc, c);
+        for (int i = 0; i < 4; ++i)
+          if (v[i]) atomicAdd(m + M_TOT + i, v[i]);
+      }
+    }
+  }
+  cluster_or_cta_sync(cs);
+}
+
 // Key sources -----------------------------------------------------------------
+// stream(): computes the keys of items j < n (token tok(j)) and calls
+//   f(valid, j, key, score) on every thread for every item slot it owns; valid
+//   is false for slots past n and, when several lanes share a label row, on all
+//   but the row's first lane.  Every lane makes the same calls.
 
 // Keys from precomputed fp32 scores [BH, T].
 struct ScoresSource {
   const float* scores;
-  __device__ __forceinline__ void fill(int bh, int T, int c0, int len, uint32_t* keys,
-                                       uint32_t* hist) const {
-    const float* src = scores + (size_t)bh * T + c0;
-    int i = threadIdx.x;
-    for (; i + 3 * kTopkThreads < len; i += 4 * kTopkThreads) {
-      float f[4];
+  __device__ __forceinline__ void prepare(int, float*) const {}
+  __device__ __forceinline__ float* scores_out(int, int) const { return nullptr; }
+  template <class Tok, class F>
+  __device__ __forceinline__ void stream(int bh, int T, int n, Tok tok, F&& f,
+                                         const float*) const {
+    const float* src = scores + (size_t)bh * T;
+    constexpr int kU = 8, kStep = kU * kTopkThreads;
+    float v[kU];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) f[u] = __ldcs(src + i + u * kTopkThreads);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t key = order_key(f[u]);
-        keys[i + u * kTopkThreads] = key;
-        atomicAdd(&hist[key >> digit_shift(0)], 1u);
-      }
+    for (int u = 0; u < kU; ++u) {
+      const int j = threadIdx.x + u * kTopkThreads;
+      v[u] = j < n ? __ldcs(src + tok(j)) : 0.f;
     }
-    for (; i < len; i += kTopkThreads) {
-      const uint32_t key = order_key(__ldcs(src + i));
-      keys[i] = key;
-      atomicAdd(&hist[key >> digit_shift(0)], 1u);
+    for (int base = 0; base < n; base += kStep) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const float x = v[u];
+        const int jn = base + kStep + threadIdx.x + u * kTopkThreads;
+        if (jn < n) v[u] = __ldcs(src + tok(jn));
+        const int j = base + threadIdx.x + u * kTopkThreads;
+        f(j < n, j, order_key(x), x);
+      }
     }
   }
 };
 
 // Keys computed from the label cache: the fused score + select path.  Scores
-// are computed exactly as k_score_vec computes them.
+// are computed exactly as k_score_vec computes them (same order of fp32
+// operations), r/8 lanes per row so that every warp load reads 512 contiguous
+// bytes, with the next slice's loads in flight while a slice is consumed.
 template <int R>
 struct LabelSource {
   const uint16_t* Q;
   const int32_t* C;
   const uint16_t* label;
-  float* scores_out;  // optional
+  float* scores;  // optional output
   int Hq, T_cap;
-  static constexpr int kChunks = R / 8;
-  static constexpr int kRows = kChunks >= 4 ? 1 : 4 / kChunks;
+  static constexpr int kLanes = R / 8;
+  static constexpr int kRowsPerInstr = 32 / kLanes;
+  static constexpr int kSlots = 4;
+  static constexpr int kStep = kTopkWarps * kSlots * kRowsPerInstr;  // items per slice
 
-  __device__ __forceinline__ void fill(int bh, int T, int c0, int len, uint32_t* keys,
-                                       uint32_t* hist) const {
-    __shared__ __align__(16) float qs[R];
+  __device__ __forceinline__ void prepare(int bh, float* qs) const {
     load_qc(Q, C, bh, bh % Hq, R, qs);
-    __syncthreads();
-    const uint4* lab = reinterpret_cast<const uint4*>(label + ((size_t)bh * T_cap + c0) * R);
-    float* out = scores_out ? scores_out + (size_t)bh * T + c0 : nullptr;
-    for (int base = 0; base < len; base += kTopkThreads * kRows) {
-      uint4 v[kRows][kChunks];
+  }
+  __device__ __forceinline__ float* scores_out(int bh, int T) const {
+    return scores ? scores + (size_t)bh * T : nullptr;
+  }
+  __device__ __forceinline__ int slot_item(int base, int i) const {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    return base + (warp * kSlots + i) * kRowsPerInstr + lane / kLanes;
+  }
+  // Rolling buffer: slot i of the next slice is loaded as soon as slot i of
+  // this slice has been taken, so kSlots loads stay in flight per thread.
+  template <class Tok, class F>
+  __device__ __forceinline__ void stream(int bh, int, int n, Tok tok, F&& f,
+                                         const float* qs) const {
+    const uint4* lab = reinterpret_cast<const uint4*>(label + (size_t)bh * T_cap * R);
+    const int chunk = (threadIdx.x & 31) % kLanes;
+    uint4 v[kSlots];
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const int t = base + threadIdx.x + i * kTopkThreads;
-        if (t < len) {
+    for (int i = 0; i < kSlots; ++i) {
+      const int j = slot_item(0, i);
+      if (j < n) v[i] = ldg_stream(lab + (size_t)tok(j) * kLanes + chunk);
+    }
+    for (int base = 0; base < n; base += kStep) {
 #pragma unroll
-          for (int c = 0; c < kChunks; ++c) v[i][c] = ldg_stream(lab + (size_t)t * kChunks + c);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const int t = base + threadIdx.x + i * kTopkThreads;
-        if (t < len) {
-          const float s = row_score<R>(v[i], qs);
-          if (out) out[t] = s;
-          const uint32_t key = order_key(s);
-          keys[t] = key;
-          atomicAdd(&hist[key >> digit_shift(0)], 1u);
-        }
+      for (int i = 0; i < kSlots; ++i) {
+        const uint4 x = v[i];
+        const int jn = slot_item(base + kStep, i);
+        if (jn < n) v[i] = ldg_stream(lab + (size_t)tok(jn) * kLanes + chunk);
+        const int j = slot_item(base, i);
+        const float s = lane_group_score<R>(x, qs, chunk);  // all lanes take part
+        f(j < n && chunk == 0, j, order_key(s), s);
       }
     }
   }
 };
 
-// grid (CS, BH), cluster (CS, 1, 1).  chunk: tokens per CTA.
+// Keys of rank r1 and r2 (1 = largest; 0 = not wanted) among keys[0..m), by a
+// three-digit radix select.  hist already holds the digit-0 histogram; hist2
+// has room for two 2048-bin histograms.
+__device__ __forceinline__ void sample_ranks(const uint32_t* keys, int m, const uint32_t* hist,
+                                             uint32_t* hist2, uint32_t* misc, uint32_t r1,
+                                             uint32_t r2, uint32_t& key1, uint32_t& key2) {
+  uint32_t* scratch = misc + 48;
+  uint32_t p1 = 0, p2 = 0;
+  for (int d = 0; d < 3; ++d) {
+    const int nb = digit_bins(d);
+    const uint32_t* h1 = hist;
+    const uint32_t* h2 = hist;
+    if (d > 0) {
+      for (int i = threadIdx.x; i < 2 * nb; i += kTopkThreads) hist2[i] = 0u;
+      __syncthreads();
+      const int hs = digit_shift(d - 1), sh = digit_shift(d);
+      for (int i = threadIdx.x; i < m; i += kTopkThreads) {
+        const uint32_t key = keys[i];
+        if (r1 && (key >> hs) == p1) atomicAdd(&hist2[(key >> sh) & (nb - 1)], 1u);
+        if (r2 && (key >> hs) == p2) atomicAdd(&hist2[nb + ((key >> sh) & (nb - 1))], 1u);
+      }
+      __syncthreads();
+      h1 = hist2;
+      h2 = hist2 + nb;
+    }
+    find_bin(h1, nb, r1, scratch, misc + M_BIN);
+    find_bin(h2, nb, r2, scratch, misc + M_BIN2);
+    if (r1) {
+      p1 = (p1 << digit_bits(d)) | misc[M_BIN];
+      r1 -= misc[M_ABOVE];
+    }
+    if (r2) {
+      p2 = (p2 << digit_bits(d)) | misc[M_BIN2];
+      r2 -= misc[M_ABOVE2];
+    }
+    __syncthreads();
+  }
+  key1 = p1;
+  key2 = p2;
+}
+
+// The streaming passes of the kernel below.
+
+// Sample pass: keys of the m sampled tokens into keys[], their digit-0
+// histogram into hist; scores of this CTA's tokens when the whole head is the
+// sample.
 template <class Source>
-__global__ void __launch_bounds__(kTopkThreads)
+__device__ __forceinline__ void sample_pass(const Source& src, int bh, int T, int m, bool whole,
+                                         uint32_t* keys, uint32_t* hist, float* scores_out,
+                                         int c0, int len, const float* qs) {
+  const int q32 = T >> 5;
+  auto tok = [whole, q32](int j) {
+    return whole ? j : ((int)((long long)(j >> 5) * q32 / kSampleBlocks) << 5) + (j & 31);
+  };
+  src.stream(bh, T, m, tok,
+             [&](bool v, int j, uint32_t key, float s) {
+               if (v) {
+                 keys[j] = key;
+                 atomicAdd(&hist[key >> digit_shift(0)], 1u);
+                 if (whole && scores_out && j >= c0 && j < c0 + len) scores_out[j] = s;
+               }
+             },
+             qs);
+}
+
+// Main pass over this CTA's tokens against the bracket [lo, hi].
+template <class Source>
+__device__ __forceinline__ void classify_pass(const Source& src, int bh, int T, int c0, int len,
+                                           uint32_t lo, uint32_t hi, float* scores_out,
+                                           uint32_t* gtm, uint32_t* eqm, uint32_t* cand_key,
+                                           uint32_t* cand_tok, uint32_t* ncand,
+                                           const float* qs) {
+  const bool one = lo == hi;
+  auto tok = [c0](int j) { return c0 + j; };
+  src.stream(bh, T, len, tok,
+             [&](bool v, int j, uint32_t key, float s) {
+               if (!v) return;
+               if (scores_out) scores_out[c0 + j] = s;
+               const uint32_t bit = 1u << (j & 31);
+               if (key > hi) {
+                 atomicOr(&gtm[j >> 5], bit);
+               } else if (key >= lo) {
+                 if (one) {
+                   atomicOr(&eqm[j >> 5], bit);
+                 } else {
+                   const uint32_t slot = atomicAdd(ncand, 1u);
+                   if (slot < kCandCap) {
+                     cand_key[slot] = key;
+                     cand_tok[slot] = (uint32_t)j;
+                   }
+                 }
+               }
+             },
+             qs);
+}
+
+// Refinement pass: histogram of digit d of this CTA's keys that carry the
+// prefix pf of the digits above d.
+template <class Source>
+__device__ __forceinline__ void digit_hist_pass(const Source& src, int bh, int T, int c0, int len,
+                                             int d, uint32_t pf, uint32_t* hist,
+                                             const float* qs) {
+  const int hs = d > 0 ? digit_shift(d - 1) : 0;
+  const int sh = digit_shift(d);
+  const uint32_t mask = (uint32_t)digit_bins(d) - 1u;
+  auto tok = [c0](int j) { return c0 + j; };
+  src.stream(bh, T, len, tok,
+             [&](bool v, int, uint32_t key, float) {
+               if (v && (d == 0 || (key >> hs) == pf)) atomicAdd(&hist[(key >> sh) & mask], 1u);
+             },
+             qs);
+}
+
+// grid (CS, BH), cluster (CS, 1, 1).  chunk: tokens per CTA, a multiple of 32.
+template <class Source>
+__global__ void __launch_bounds__(kTopkThreads, 3)  // three CTAs per SM: up to 85 registers
 k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
   extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t* hist = sm + TopkSmem::kHist;
-  uint32_t* scratch = sm + TopkSmem::kScan;
-  uint32_t* misc = sm + TopkSmem::kMisc;
-  uint32_t* keys = sm + TopkSmem::kKeys;
-
   const int cs = gridDim.x;
   const int rank = blockIdx.x;  // == cluster rank: the cluster spans grid dimension x
   const int bh = blockIdx.y;
+  const TopkLayout L(chunk, cs);
+  uint32_t* hist = sm;
+  uint32_t* misc = sm + L.small;
+  uint32_t* warp_gt = misc + 32;
+  uint32_t* warp_eq = misc + 40;
+  float* qs = reinterpret_cast<float*>(misc + 64);
+  uint32_t* gtm = sm + L.masks;
+  uint32_t* eqm = gtm + chunk / 32;
+  uint32_t* cand_key = sm + L.X;  // also the sample keys while sampling
+  uint32_t* cand_tok = cand_key + kCandCap;  // also two histograms while sampling
+
   const int c0 = min(rank * chunk, T);
   const int len = min(chunk, T - c0);
+  const int groups = (len + 31) >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* scores_out = src.scores_out(bh, T);
 
-  for (int i = threadIdx.x; i < TopkSmem::kKeys; i += kTopkThreads) sm[i] = 0u;
-  // every CTA of the cluster is running and its merged buffers are zero
-  // before any remote access
+  for (int i = threadIdx.x; i < L.small + 64; i += kTopkThreads) sm[i] = 0u;
+  for (int i = threadIdx.x; i < 2 * (chunk / 32); i += kTopkThreads) gtm[i] = 0u;
+  src.prepare(bh, qs);
+  // every CTA of the cluster is running and its counters are zero before any
+  // remote access
   cluster_or_cta_sync(cs);
 
-  src.fill(bh, T, c0, len, keys, hist);
+  // ---- 1. sample ---------------------------------------------------------------
+  const bool whole = T <= kSample;
+  const int m = whole ? T : kSample;
+  sample_pass(src, bh, T, m, whole, cand_key, hist, scores_out, c0, len, qs);
   __syncthreads();
 
-  uint32_t krem = (uint32_t)k, prefix = 0u, thr = 0u, need = 0u;
-  bool ge_mode = false;
+  // ---- 2. bracket ----------------------------------------------------------------
+  uint32_t lo, hi;
+  if (whole) {
+    uint32_t thr, unused;
+    sample_ranks(cand_key, m, hist, cand_tok, misc, (uint32_t)k, 0u, thr, unused);
+    lo = hi = thr;
+  } else {
+    const float e = (float)k * (float)m / (float)T;
+    const float sd = sqrtf(e * (1.f - (float)k / (float)T));
+    const float margin = kBracketSigmas * sd + 2.f;
+    const int r_hi = (int)floorf(e - margin), r_lo = (int)ceilf(e + margin);
+    uint32_t khi, klo;
+    sample_ranks(cand_key, m, hist, cand_tok, misc, r_hi >= 1 ? (uint32_t)r_hi : 0u,
+                 r_lo <= m ? (uint32_t)r_lo : 0u, khi, klo);
+    hi = r_hi >= 1 ? khi : 0xffffffffu;
+    lo = r_lo <= m ? klo : 0u;
+  }
 
-  for (int d = 0; d < 3; ++d) {
-    const int nbins = digit_bins(d), shift = digit_shift(d);
-    if (d > 0) {
-      // local histogram of digit d over the keys that carry the chosen prefix
-      for (int i = threadIdx.x; i < nbins; i += kTopkThreads) hist[i] = 0u;
-      __syncthreads();
-      const int hi_shift = digit_shift(d - 1);
-      for (int i = threadIdx.x; i < len; i += kTopkThreads) {
-        const uint32_t key = keys[i];
-        if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
+  // ---- 3/4. stream and check; exact refinement if the bracket fails -----------
+  int level = 0;  // refinement digits done
+  uint32_t prefix = 0, krem = (uint32_t)k;
+  for (;;) {
+    const bool one = lo == hi;
+    if (whole) {
+      // every key of the head is in cand_key (the sample): this CTA's range;
+      // the bracket is exact here, so no candidate is listed over them
+      for (int j = threadIdx.x; j < len; j += kTopkThreads) {
+        const uint32_t key = cand_key[c0 + j];
+        if (key > hi) atomicOr(&gtm[j >> 5], 1u << (j & 31));
+        else if (key == hi) atomicOr(&eqm[j >> 5], 1u << (j & 31));
       }
-      __syncthreads();
+    } else {
+      classify_pass(src, bh, T, c0, len, lo, hi, level == 0 ? scores_out : nullptr, gtm, eqm,
+                    cand_key, cand_tok, &misc[M_NCAND], qs);
     }
-    const uint32_t* merged = hist;
-    if (cs > 1) {
-      cg::cluster_group cl = cg::this_cluster();
-      uint32_t* m0 = cl.map_shared_rank(sm + TopkSmem::kMerged0 + d * 2048, 0);
-      for (int i = threadIdx.x; i < nbins; i += kTopkThreads) {
-        const uint32_t v = hist[i];
-        if (v) atomicAdd(m0 + i, v);
-      }
-      cl.sync();
-      merged = m0;
+    __syncthreads();
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int g = threadIdx.x; g < groups; g += kTopkThreads) {
+      n_gt += __popc(gtm[g]);
+      n_eq += __popc(eqm[g]);
     }
-    find_bin(merged, nbins, krem, scratch, misc);
-    const uint32_t bin = misc[M_BIN], above = misc[M_ABOVE], cnt = misc[M_CNT];
-    krem -= above;
-    prefix = (prefix << digit_bits(d)) | bin;
-    if (cnt == krem) {  // the whole bin is selected
-      ge_mode = true;
-      thr = prefix << shift;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
+    if (lane == 0) {
+      warp_gt[warp] = n_gt;
+      warp_eq[warp] = n_eq;
+    }
+    __syncthreads();
+    const uint32_t ncand = misc[M_NCAND];
+    uint32_t mine[4] = {0u, 0u, ncand, ncand > (uint32_t)kCandCap ? 1u : 0u};
+    for (int w = 0; w < kTopkWarps; ++w) {
+      mine[0] += warp_gt[w];
+      mine[1] += warp_eq[w];
+    }
+    cluster_totals(misc, mine, cs);
+    const uint32_t tot_gt = misc[M_TOT], tot_eq = misc[M_TOT + 1];
+    const uint32_t tot_cand = misc[M_TOT + 2], tot_ovf = misc[M_TOT + 3];
+    const bool ok = tot_ovf == 0 && tot_gt < (uint32_t)k &&
+                    (uint32_t)k <= tot_gt + (one ? tot_eq : tot_cand);
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int i = 0; i < 4; ++i) misc[M_TOT + i] = 0u;  // before the next cluster barrier
+    if (ok) {
+      krem = (uint32_t)k - tot_gt;
       break;
     }
-    if (d == 2) {
-      thr = prefix;
-      need = krem;
-    }
+
+    // Exact refinement.  The rank sought within the current bracket: k itself
+    // while no prefix is fixed (the failed bracket came from the sample), else
+    // k minus the keys above the prefix's range.
+    krem = level == 0 ? (uint32_t)k : (uint32_t)k - tot_gt;
+    const int d = level;
+    for (int i = threadIdx.x; i < 2048; i += kTopkThreads) hist[i] = 0u;
+    if (cs > 1)
+      for (int i = threadIdx.x; i < 4096; i += kTopkThreads) sm[L.merged0 + i] = 0u;
+    for (int i = threadIdx.x; i < 2 * (chunk / 32); i += kTopkThreads) gtm[i] = 0u;
+    if (threadIdx.x == 0) misc[M_NCAND] = 0u;
+    // every CTA has zeroed its merged copies before anyone adds into them
+    cluster_or_cta_sync(cs);
+    digit_hist_pass(src, bh, T, c0, len, d, prefix, hist, qs);
+    __syncthreads();
+    const uint32_t* h =
+        cluster_hist(hist, sm + (d == 1 ? L.merged1 : L.merged0), digit_bins(d), cs);
+    find_bin(h, digit_bins(d), krem, misc + 48, misc + M_BIN);
+    prefix = (prefix << digit_bits(d)) | misc[M_BIN];
+    ++level;
+    lo = prefix << digit_shift(d);
+    hi = lo | ((1u << digit_shift(d)) - 1u);
+    __syncthreads();
   }
 
-  // ---- output: counts per warp --------------------------------------------
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = ((len + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
-  const int w0 = min(warp * seg, len), w1 = min(w0 + seg, len);
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int i = w0 + lane; i - lane < w1; i += 32) {
-    const bool in = i < w1;
-    const uint32_t key = in ? keys[i] : 0u;
-    const bool gt = in && (ge_mode ? key >= thr : key > thr);
-    const bool eq = in && !ge_mode && key == thr;
-    n_gt += __popc(__ballot_sync(0xffffffffu, gt));
-    n_eq += __popc(__ballot_sync(0xffffffffu, eq));
+  // ---- 5. resolve within the bracket -------------------------------------------
+  uint32_t need = krem;
+  if (lo != hi) {
+    const uint32_t ncand = misc[M_NCAND];
+    uint32_t p = 0, r = krem;
+    for (int d = 0; d < 3; ++d) {
+      const int nb = digit_bins(d);
+      uint32_t* mg = sm + (d == 1 ? L.merged1 : L.merged0);
+      for (int i = threadIdx.x; i < nb; i += kTopkThreads) hist[i] = 0u;
+      if (cs > 1)
+        for (int i = threadIdx.x; i < nb; i += kTopkThreads) mg[i] = 0u;
+      cluster_or_cta_sync(cs);
+      const int hs = d > 0 ? digit_shift(d - 1) : 0;
+      for (uint32_t s = threadIdx.x; s < ncand; s += kTopkThreads) {
+        const uint32_t key = cand_key[s];
+        if (d == 0 || (key >> hs) == p) atomicAdd(&hist[(key >> digit_shift(d)) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+      const uint32_t* h = cluster_hist(hist, mg, nb, cs);
+      find_bin(h, nb, r, misc + 48, misc + M_BIN);
+      p = (p << digit_bits(d)) | misc[M_BIN];
+      r -= misc[M_ABOVE];
+      __syncthreads();
+    }
+    need = r;
+    for (uint32_t s = threadIdx.x; s < ncand; s += kTopkThreads) {
+      const uint32_t key = cand_key[s], j = cand_tok[s];
+      if (key > p)
+        atomicOr(&gtm[j >> 5], 1u << (j & 31));
+      else if (key == p)
+        atomicOr(&eqm[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
   }
-  if (lane == 0) {
-    sm[TopkSmem::kWarpGt + warp] = n_gt;
-    sm[TopkSmem::kWarpEq + warp] = n_eq;
+
+  // ---- 6. counts, cluster prefix, write ------------------------------------------
+  const int gpw = (groups + kTopkWarps - 1) / kTopkWarps;
+  const int g0 = min(warp * gpw, groups), g1 = min(g0 + gpw, groups);
+  {
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int g = g0 + lane; g < g1; g += 32) {
+      n_gt += __popc(gtm[g]);
+      n_eq += __popc(eqm[g]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
+    if (lane == 0) {
+      warp_gt[warp] = n_gt;
+      warp_eq[warp] = n_eq;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t g = 0, e = 0;
+    uint32_t a = 0, e = 0;
     for (int w = 0; w < kTopkWarps; ++w) {
-      g += sm[TopkSmem::kWarpGt + w];
-      e += sm[TopkSmem::kWarpEq + w];
+      a += warp_gt[w];
+      e += warp_eq[w];
     }
-    misc[M_CTA_GT] = g;
-    misc[M_CTA_EQ] = e;
+    if (cs > 1) {  // push this CTA's counts into every later CTA of the cluster
+      cg::cluster_group cl = cg::this_cluster();
+      for (int c = rank + 1; c < cs; ++c) {
+        uint32_t* mm = cl.map_shared_rank(misc, c);
+        atomicAdd(mm + M_GT_BEFORE, a);
+        atomicAdd(mm + M_EQ_BEFORE, e);
+      }
+    }
   }
   cluster_or_cta_sync(cs);
 
-  // counts of the CTAs before this one in the cluster, then of earlier warps
-  uint32_t gt_before = 0, eq_before = 0;
-  if (cs > 1) {
-    cg::cluster_group cl = cg::this_cluster();
-    for (int c = 0; c < rank; ++c) {
-      const uint32_t* m = cl.map_shared_rank(misc, c);
-      gt_before += m[M_CTA_GT];
-      eq_before += m[M_CTA_EQ];
-    }
-  }
+  uint32_t gt_before = misc[M_GT_BEFORE], eq_before = misc[M_EQ_BEFORE];
   for (int w = 0; w < warp; ++w) {
-    gt_before += sm[TopkSmem::kWarpGt + w];
-    eq_before += sm[TopkSmem::kWarpEq + w];
+    gt_before += warp_gt[w];
+    eq_before += warp_eq[w];
   }
 
-  // ---- output: place the selected indices ----------------------------------
+  // 32 groups per step, one per lane; warp scans give each group its first tie
+  // rank and its first output position.
   uint32_t tie = eq_before;
   uint32_t out = gt_before + min(eq_before, need);
   int32_t* dst = idx + (size_t)bh * k;
-  const uint32_t lt = lanemask_lt();
-  for (int i = w0 + lane; i - lane < w1; i += 32) {
-    const bool in = i < w1;
-    const uint32_t key = in ? keys[i] : 0u;
-    const bool gt = in && (ge_mode ? key >= thr : key > thr);
-    const bool eq = in && !ge_mode && key == thr;
-    const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && tie + __popc(eq_mask & lt) < need);
-    const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
-    const uint32_t pos = out + __popc(sel_mask & lt);
-    if (sel && pos < (uint32_t)k) dst[pos] = c0 + i;
-    tie += __popc(eq_mask);
-    out += __popc(sel_mask);
+  for (int base = g0; base < g1; base += 32) {
+    const int g = base + lane;
+    const uint32_t gmask = g < g1 ? gtm[g] : 0u;
+    const uint32_t emask = g < g1 ? eqm[g] : 0u;
+    const uint32_t ne = __popc(emask);
+    uint32_t ne_incl = ne;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, ne_incl, o);
+      if (lane >= o) ne_incl += v;
+    }
+    const uint32_t my_tie = tie + ne_incl - ne;
+    const uint32_t take = need > my_tie ? min(need - my_tie, ne) : 0u;  // ties kept here
+    uint32_t takem = emask;  // the first `take` set bits of emask
+    if (take < ne) {
+      uint32_t rest = emask;
+      for (uint32_t j = 0; j < take; ++j) rest &= rest - 1u;
+      takem = emask ^ rest;
+    }
+    uint32_t selm = gmask | takem;
+    const uint32_t n = __popc(selm);
+    uint32_t n_incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, n_incl, o);
+      if (lane >= o) n_incl += v;
+    }
+    uint32_t pos = out + n_incl - n;
+    while (selm) {
+      const int b = __ffs(selm) - 1;
+      selm &= selm - 1u;
+      if (pos < (uint32_t)k) dst[pos] = c0 + g * 32 + b;
+      ++pos;
+    }
+    tie += __shfl_sync(0xffffffffu, ne_incl, 31);
+    out += __shfl_sync(0xffffffffu, n_incl, 31);
   }
-  // no CTA leaves while another may still read its shared memory
-  cluster_or_cta_sync(cs);
 }
 
 }  // namespace ds

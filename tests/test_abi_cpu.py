@@ -99,7 +99,7 @@ def test_bad_sizes_and_pointers():
     assert lib.ds_topk(P, P, 0, 10, 1, NUL, 0, NUL) == bad
     assert lib.ds_topk(NUL, P, 4, 10, 1, NUL, 0, NUL) == bad
     assert lib.ds_topk(P, mis, 4, 10, 1, NUL, 0, NUL) == bad
-    assert lib.ds_topk(P, P, 4, 16 * 40960 + 1, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_topk(P, P, 4, 16 * 65536 + 1, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
     assert lib.ds_topk(P, P, 70000, 10, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
     # fused score+topk: r not a multiple of 8 needs a score buffer
     assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 20, NUL) == bad

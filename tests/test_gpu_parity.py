@@ -143,6 +143,7 @@ def _check_topk(scores: np.ndarray, k: int):
 
 
 TOPK_SHAPES = [(1, 1, 1), (3, 7, 2), (5, 64, 64), (2, 65, 10), (1, 4096, 256), (7, 1000, 999),
+               (1, 786432, 49152), (4, 32768, 32768), (40, 40000, 1000),
                (1, 40961, 5000), (2, 100000, 6250), (64, 100000, 100), (1, 262144, 16384),
                (1, 655360, 40960), (300, 32768, 2048)]
 
@@ -377,3 +378,47 @@ def test_full_workload_sampled_heads(name):
             assert set(pos[h].tolist()) <= set(I[0, h].tolist())
     print(f"{name}: max abs err sparse {worst['sparse']:.3g} dense {worst['dense']:.3g}")
     inp.free()
+
+
+@pytest.mark.parametrize("B,H,T,k", [(1, 2, 5000, 1234), (2, 3, 70000, 20000)])
+def test_score_topk_all_scores_tied(B, H, T, k):
+    """Every K row identical: all scores tie, the first k tokens must be kept.
+
+    Exercises the path where one CTA has more candidates than it can list and
+    recomputes their exact keys from the label cache."""
+    w = dsgen.Workload("tied", B=B, Hq=H, Hkv=H, T=T, r=16, k=k, n_out=16, seed=4242)
+    inp = gu.Inputs(w, with_v=False)
+    inp.dK[:] = inp.dK[:, :, :1, :]
+    label = _label_dev(inp, T)
+    idx = torch.empty((B * H, k), dtype=torch.int32, device="cuda")
+    ds.score_topk(inp.dQ, inp.dC, label, idx, T)
+    want = torch.arange(k, dtype=torch.int32, device="cuda").expand(B * H, -1)
+    assert torch.equal(idx, want)
+
+
+def _sampled_tokens(T):
+    """Tokens the top-k draws its bracketing sample from (128 blocks of 32)."""
+    q = T // 32
+    starts = [(b * q // 128) * 32 for b in range(128)]
+    return np.concatenate([np.arange(s, s + 32) for s in starts])
+
+
+@pytest.mark.parametrize("k", [50000, 49999, 1, 99999])
+def test_topk_bracket_overflow_falls_back_exactly(k):
+    """Two-valued scores: the sample bracket holds every token, the candidate lists
+    overflow and the exact refinement path must produce the exact top-k."""
+    T = 100000
+    rng = np.random.default_rng(k)
+    s = np.where(rng.random((2, T)) < 0.5, 1.0, -1.0).astype(np.float32)
+    _check_topk(s, k)
+
+
+@pytest.mark.parametrize("k", [1000, 4096, 10000])
+def test_topk_bracket_miss_falls_back_exactly(k):
+    """The sampled blocks score higher than every other token, so the sample
+    misplaces the k-th key; the result must still be exact."""
+    T = 100000
+    rng = np.random.default_rng(k + 7)
+    s = rng.standard_normal((2, T)).astype(np.float32)
+    s[:, _sampled_tokens(T)] = 100.0
+    _check_topk(s, k)
