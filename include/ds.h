@@ -82,7 +82,8 @@ enum {
 /* Device status bits (ds_device_status). */
 enum {
   DS_DEV_BAD_CHANNEL = 1u, /* a channel id in C was outside [0, d); masked  */
-  DS_DEV_BAD_INDEX = 2u    /* a token index was outside [0, T); clamped     */
+  DS_DEV_BAD_INDEX = 2u,   /* a token index was outside [0, T); clamped     */
+  DS_DEV_TIMEOUT = 4u      /* a bounded wait on an asynchronous copy gave up  */
 };
 
 /*
@@ -156,7 +157,9 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
  * entries in [0, T) (out-of-range entries are clamped and flagged);
  * O: [B,Hq,d] fp32; lse: [B,Hq] fp32 or NULL.  Requires 1 <= k <= T <= T_cap.
  * ws: ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k) bytes of device
- * memory (contents need not be initialised; may be NULL when that size is 0).
+ * memory, zero-filled before its first use (it holds per-head counters that
+ * every call leaves at zero again); may be NULL when that size is 0.  Calls
+ * that may overlap on the GPU need separate workspaces.
  */
 ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
                            float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
@@ -167,7 +170,7 @@ ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const in
  * token sparsity accelerates (Double Sparsity page, Experimental highlights:
  * attention-operation speed-up).  Same as ds_sparse_decode with
  * idx = 0..T-1 for every head.  ws: ds_workspace_size(DS_OP_DECODE, dims, T,
- * T) bytes.
+ * T) bytes, zero-filled before first use as for ds_sparse_decode.
  */
 ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float* lse,
                     ds_dims dims, int32_t T, float scale, void* ws, size_t ws_bytes,
@@ -198,9 +201,10 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
  * The first call on each device looks up the array's device address with
  * that device current (cudaGetSymbolAddress); make that first call outside
  * any stream capture.  All calls on a device share the one array and it keeps
- * the previous call's contents (nothing in it needs to start at zero): calls
- * that may overlap on the GPU -- on different streams without an ordering
- * between them -- race on it and must not be issued.
+ * the previous call's contents; each call first clears (on `stream`) the
+ * per-head counters that must start at zero.  Calls that may overlap on the
+ * GPU -- on different streams without an ordering between them -- race on the
+ * array and must not be issued.
  */
 #define DS_NOALLOC_SCRATCH_BYTES (4u << 20)
 ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,

@@ -130,9 +130,12 @@ def workspace_size(op: int, dims: Dims, T: int, k: int) -> int:
 
 
 def workspace(op: int, dims: Dims, T: int, k: int, device) -> torch.Tensor | None:
-    """A device buffer of the size ``op`` needs (None when it needs none)."""
+    """A zero-filled device buffer of the size ``op`` needs (None when it needs none).
+
+    Calls leave the workspace zero-filled again, so one buffer serves any number
+    of calls that do not overlap on the GPU."""
     n = workspace_size(op, dims, T, k)
-    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
 
 
 # ---------------------------------------------------------------------------

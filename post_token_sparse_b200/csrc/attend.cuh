@@ -18,7 +18,8 @@
 // wait.  Per row: 16 FMAs + 3 xor-shuffles for the logit, an online-softmax
 // update (running max m, sum l, log2 domain), 16 FMAs into the accumulator.
 // Warps then merge through shared memory; with S > 1 each split writes
-// (m, l, unnormalised o) and k_lse_merge combines them.
+// (m, l, unnormalised o) to the workspace and the head's last split to finish
+// (found by an arrival counter) combines them.
 #pragma once
 
 #include "common.cuh"
@@ -27,7 +28,7 @@ namespace ds {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kAttnStages = 8;
+constexpr int kAttnStages = 4;
 constexpr int kAttnStageU4 = 4 * 32;  // 4 rows x (16 uint4 of K + 16 uint4 of V) = 2 KB
 constexpr int kPartialStride = 132;   // floats per split partial: m, l, pad, pad, o[128]
 constexpr int kMaxRowsPerSplitSparse = 2048;
@@ -39,7 +40,8 @@ struct AttnParams {
   const int32_t* idx;  // null: dense (rows 0..T-1)
   float* O;
   float* lse;      // optional
-  float* partial;  // [BH, S, kPartialStride] when S > 1
+  float* partial;      // [BH, S, kPartialStride] when S > 1
+  uint32_t* arrivals;  // [BH] split-arrival counters (zero between calls) when S > 1
   int Hq, Hkv, T_cap, T;
   int rows;           // k (sparse) or T (dense)
   int rows_per_split; // multiple of 4
@@ -229,32 +231,35 @@ k_attend(const AttnParams p) {
     p.O[(size_t)bh * kHeadDim + j] = o / L;
     if (p.lse && j == 0) p.lse[bh] = (M + log2f(L)) * 0.69314718055994530942f;
   } else {
+    // publish this split's partial; the last split of the head to arrive
+    // merges all of them and resets the head's counter for the next call
     float* part = p.partial + ((size_t)bh * S + split) * kPartialStride;
     part[4 + j] = o;
     if (j == 0) {
       part[0] = M;
       part[1] = L;
     }
+    __threadfence();
+    __syncthreads();
+    __shared__ uint32_t last;
+    if (j == 0) last = atomicAdd(&p.arrivals[bh], 1u) == (uint32_t)(S - 1);
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      const float* all = p.partial + (size_t)bh * S * kPartialStride;
+      float Mg = -INFINITY;
+      for (int s = 0; s < S; ++s) Mg = fmaxf(Mg, __ldcg(all + s * kPartialStride));
+      float Lg = 0.f, og = 0.f;
+      for (int s = 0; s < S; ++s) {
+        const float a = rescale(__ldcg(all + s * kPartialStride), Mg);
+        Lg = fmaf(__ldcg(all + s * kPartialStride + 1), a, Lg);
+        og = fmaf(__ldcg(all + s * kPartialStride + 4 + j), a, og);
+      }
+      p.O[(size_t)bh * kHeadDim + j] = og / Lg;
+      if (p.lse && j == 0) p.lse[bh] = (Mg + log2f(Lg)) * 0.69314718055994530942f;
+      if (j == 0) p.arrivals[bh] = 0u;
+    }
   }
-}
-
-// Combine S split partials per head: O = sum_s 2^(m_s-M) o_s / sum_s 2^(m_s-M) l_s.
-// grid BH, block 128 (thread j = dim j).
-__global__ void __launch_bounds__(kHeadDim)
-k_lse_merge(const float* __restrict__ partial, float* __restrict__ O, float* __restrict__ lse,
-            int S) {
-  const int bh = blockIdx.x, j = threadIdx.x;
-  const float* part = partial + (size_t)bh * S * kPartialStride;
-  float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, part[s * kPartialStride]);
-  float L = 0.f, o = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float a = rescale(part[s * kPartialStride], M);
-    L = fmaf(part[s * kPartialStride + 1], a, L);
-    o = fmaf(part[s * kPartialStride + 4 + j], a, o);
-  }
-  O[(size_t)bh * kHeadDim + j] = o / L;
-  if (lse && j == 0) lse[bh] = (M + log2f(L)) * 0.69314718055994530942f;
 }
 
 }  // namespace ds

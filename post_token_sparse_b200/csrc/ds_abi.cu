@@ -53,12 +53,13 @@ ds_status check_dims(const ds_dims& d) {
 }
 
 // ---- split plan for the attention kernels (device independent) -------------
-// Heads are cut into S splits of rows_per_split rows so that the grid has
-// about kTargetCtas CTAs, no split is smaller than kMinRowsPerSplit rows
-// unless the head itself is, and sparse splits fit their index list in
-// shared memory.
-constexpr int kTargetCtas = 148 * 4;
-constexpr int kMinRowsPerSplit = 128;
+// Heads are cut into S splits of rows_per_split rows.  S is the smallest count
+// (splits of at least kMinRowsPerSplit rows; sparse splits keep their index
+// list in shared memory, so at most kMaxRowsPerSplitSparse rows) whose grid
+// fills its last wave of kWaveCtas CTAs (148 SMs x 6 resident CTAs) to within
+// 10%, else the one that fills it best.
+constexpr int kWaveCtas = 148 * 6;
+constexpr int kMinRowsPerSplit = 64;
 
 struct SplitPlan {
   int S;
@@ -66,19 +67,29 @@ struct SplitPlan {
 };
 
 SplitPlan plan_splits(int heads, int rows, bool sparse) {
-  int S = (kTargetCtas + heads - 1) / heads;
-  S = std::min(S, (rows + kMinRowsPerSplit - 1) / kMinRowsPerSplit);
-  if (sparse) S = std::max(S, (rows + kMaxRowsPerSplitSparse - 1) / kMaxRowsPerSplitSparse);
-  S = std::max(S, 1);
-  int rps = (rows + S - 1) / S;
+  const int s_min = sparse ? (rows + kMaxRowsPerSplitSparse - 1) / kMaxRowsPerSplitSparse : 1;
+  const int s_max = std::max(s_min, std::min(256, rows / kMinRowsPerSplit));
+  int best = s_min;
+  double best_waste = 1e30;
+  for (int S = s_min; S <= s_max; ++S) {
+    const double n = (double)heads * S;
+    const double waves = std::ceil(n / kWaveCtas);
+    const double waste = waves * kWaveCtas / n;  // >= 1; 1 = the last wave is full
+    if (waste < best_waste - 1e-9) {
+      best_waste = waste;
+      best = S;
+    }
+    if (waste <= 1.10) break;
+  }
+  int rps = (rows + best - 1) / best;
   rps = (rps + 3) & ~3;
-  S = (rows + rps - 1) / rps;
-  return {S, rps};
+  return {(rows + rps - 1) / rps, rps};
 }
 
+// Workspace: the split partials, then one arrival counter per head.
 size_t partial_bytes(int heads, const SplitPlan& sp) {
   if (sp.S <= 1) return 0;
-  size_t b = (size_t)heads * sp.S * kPartialStride * sizeof(float);
+  size_t b = (size_t)heads * sp.S * kPartialStride * sizeof(float) + (size_t)heads * 4;
   return (b + 255) & ~size_t(255);
 }
 
@@ -241,6 +252,9 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
   p.O = O;
   p.lse = lse;
   p.partial = static_cast<float*>(ws);
+  p.arrivals = ws ? reinterpret_cast<uint32_t*>(static_cast<float*>(ws) +
+                                                (size_t)BH * sp.S * kPartialStride)
+                  : nullptr;
   p.Hq = d.Hq;
   p.Hkv = d.Hkv;
   p.T_cap = d.T_cap;
@@ -255,9 +269,6 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
     k_attend<true><<<grid, kAttnThreads, smem, st>>>(p);
   else
     k_attend<false><<<grid, kAttnThreads, smem, st>>>(p);
-  ds_status s = launched();
-  if (s != DS_OK || sp.S == 1) return s;
-  k_lse_merge<<<BH, kHeadDim, 0, st>>>(p.partial, O, lse, sp.S);
   return launched();
 }
 
@@ -463,6 +474,11 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
   if (need > 0) {
     s = noalloc_scratch(&scratch);
     if (s != DS_OK) return s;
+    // the arrival counters after the partials must start at zero
+    const size_t counters = (size_t)BH * sp.S * kPartialStride * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(scratch) + counters, 0,
+                                    (size_t)BH * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
 }

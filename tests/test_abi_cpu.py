@@ -127,11 +127,19 @@ def test_workspace_checked_before_launch():
 
 def test_workspace_sizes():
     lib = ds.lib()
-    # many heads, short rows: no split, no workspace
+    # short rows: no split, no workspace
     d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
-    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 512) == 0
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 100) == 0
     assert lib.ds_workspace_size(ds.OP_TOPK, d, 32768, 512) == 0
     assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == 0
+    # heads that fill whole waves of the grid on their own (148 SMs x 6): no split
+    d = _dims(B=8, Hq=111, Hkv=111, T_cap=32768, r=8)
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 2048) == 0
+    # otherwise the split count fills the last wave: partials + one counter per head
+    d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
+    n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 2048)
+    S = round((n - 1024 * 4) / (1024 * 132 * 4))
+    assert S >= 2 and n >= 1024 * (S * 132 * 4 + 4) and n % 256 == 0
     # long single sequence: split, 132 floats per split, 256-byte rounded
     d = _dims(B=1, Hq=32, Hkv=32, T_cap=262144, r=8)
     n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 262144, 16384)

@@ -40,7 +40,7 @@ def _raw_noalloc(Q, K, V, idx, O, lse, dims, T, k, scale):
 @pytest.mark.parametrize("B,Hq,Hkv,T,k", [
     (1, 4, 4, 50000, 20000),   # few heads, many rows: split partials in the scratch array
     (1, 8, 2, 9000, 4000),     # grouped KV heads, split
-    (8, 32, 32, 2048, 128),    # many heads, short rows: no split, no scratch used
+    (8, 32, 32, 2048, 100),    # short rows: no split, no scratch used
 ])
 def test_noalloc_matches_workspace_path_twice(B, Hq, Hkv, T, k):
     w = dsgen.Workload("noalloc", B=B, Hq=Hq, Hkv=Hkv, T=T, r=8, k=k, n_out=8, seed=900 + T)
@@ -49,7 +49,7 @@ def test_noalloc_matches_workspace_path_twice(B, Hq, Hkv, T, k):
     dims = ds.dims_of(inp.dQ, inp.dK, w.r)
     need = ds.workspace_size(ds.OP_SPARSE_DECODE, dims, T, k)
     assert need <= ds.NOALLOC_SCRATCH_BYTES
-    assert (need == 0) == (B * Hq >= 256)
+    assert (need == 0) == (k < 128)
     for call in range(2):
         idx_np = np.sort(np.stack([rng.choice(T, k, replace=False) for _ in range(B * Hq)]),
                          axis=1).astype(np.int32)
