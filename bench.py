@@ -5,8 +5,9 @@
 
 A step is the whole hot path for one decode token of every sequence in the
 batch: append the new token's label row, score every cached token on the
-label channels and keep the top k (one fused launch), then exact attention
-over the kept rows.  Inputs are seeded and synthetic (``dsgen``) and resident
+label channels and keep the top k, then exact attention over the kept rows --
+one ds_decode_step call (one launch where the sizes allow; the same step as
+separate calls is timed beside it for per-kernel stage times).  Inputs are seeded and synthetic (``dsgen``) and resident
 in HBM; the step is one CUDA graph; L2 is flushed (256 MiB written) between
 steps and each step is timed with CUDA events, so every step reads its bytes
 from HBM.
@@ -53,6 +54,9 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--unfused", action="store_true",
                    help="separate score and top-k launches instead of the fused one")
+    p.add_argument("--mode", default="step", choices=["step", "calls"],
+                   help="step: ds_decode_step; calls: label append, score+top-k and "
+                        "sparse attention as separate calls")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--batch", type=int, default=None,
                    help="override the workload's batch size (smaller captures for ncu)")
@@ -159,19 +163,23 @@ class ClockSampler:
 class Step:
     """One decode step of workload ``w`` on the current GPU, captured as a CUDA graph.
 
-    Stages: [0] label row of the new token, [1] fused score + top-k (or score
-    then top-k), [2] sparse attention (+ split merge).
+    mode "step": ds_decode_step (label row of the new token, selection and
+    attention; one launch when the sizes allow).  mode "calls": the same step as
+    separate calls, one stage each: [0] label row of the new token, [1] score +
+    top-k (fused, or score then top-k with fused=False), [2] sparse attention.
+    dense=True: ds_decode over every token.
     """
 
     STAGES = ("label_append", "score_topk", "sparse_decode")
 
     def __init__(self, w: dsgen.Workload, fused: bool = True, dense: bool = False,
-                 inputs=None):
+                 inputs=None, mode: str = "calls"):
         import torch
 
         import post_token_sparse_b200 as ds
 
         self.ds, self.torch, self.w, self.fused, self.dense = ds, torch, w, fused, dense
+        self.mode = "dense" if dense else mode
         self.Q, self.K, self.V = inputs if inputs is not None else device_inputs(w)
         self.C = torch.from_numpy(dsgen.channels(w)).cuda()
         BH = w.B * w.Hq
@@ -184,7 +192,8 @@ class Step:
             self.scores = None if fused else torch.empty((BH, w.T), dtype=torch.float32,
                                                          device="cuda")
             dims = ds.dims_of(self.Q, self.K, w.r)
-            self.ws = ds.workspace(ds.OP_SPARSE_DECODE, dims, w.T, w.k, "cuda")
+            op = ds.OP_DECODE_STEP if self.mode == "step" else ds.OP_SPARSE_DECODE
+            self.ws = ds.workspace(op, dims, w.T, w.k, "cuda")
         else:
             dims = ds.dims_of(self.Q, self.K, w.r)
             self.ws = ds.workspace(ds.OP_DECODE, dims, w.T, w.T, "cuda")
@@ -198,6 +207,10 @@ class Step:
         if self.dense:
             return [lambda: ds.decode(self.Q, self.K, self.V, self.O, w.T, w.scale, lse=self.lse,
                                       ws=self.ws)]
+        if self.mode == "step":
+            return [lambda: ds.decode_step(self.Q, self.K, self.V, self.C, self.label, self.idx,
+                                           self.O, w.T, w.scale, append=True, lse=self.lse,
+                                           ws=self.ws)]
         s0 = lambda: ds.label_append(self.K, self.C, self.label, w.T - 1, 1)  # noqa: E731
         if self.fused:
             s1 = lambda: ds.score_topk(self.Q, self.C, self.label, self.idx, w.T)  # noqa: E731
@@ -266,11 +279,13 @@ def step_bytes(w: dsgen.Workload) -> int:
 def stage_bytes(w: dsgen.Workload):
     """Algorithmic bytes per launch of each stage."""
     BH = w.B * w.Hq
-    return {
+    st = {
         "label_append": w.B * w.Hkv * w.d * 2 + BH * w.r * 2,
         "score_topk": w.label_bytes() + BH * (w.r * 2 + w.k * 4),
         "sparse_decode": w.sparse_decode_bytes(),
     }
+    st["decode_step"] = sum(st.values())
+    return st
 
 
 def time_device(step: Step, steps: int, warmup: int):
@@ -406,14 +421,19 @@ def run_reference(args, rank, world):
 
 
 def sweep_entry(w, steps, warmup, hbm_peak, fused=True, inputs=None):
-    st = Step(w, fused=fused, inputs=inputs)
-    tot, stg = time_device(st, steps, warmup)
+    """The decode step (ds_decode_step) and, beside it, the separate calls' stages."""
+    st = Step(w, fused=fused, inputs=inputs, mode="step")
+    tot, _ = time_device(st, steps, warmup)
     st.release()
     ms = tot / steps
+    sc = Step(w, fused=fused, inputs=inputs, mode="calls")
+    _, stg = time_device(sc, steps, warmup)
+    sc.release()
     sb = stage_bytes(w)
     att_ms = stg[2] / steps
     return {"us_per_step": ms * 1e3, "gbs": step_bytes(w) / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": step_bytes(w) / (ms * 1e-3) / 1e9 / hbm_peak,
+            "calls_us_per_step": sum(stg) / steps * 1e3,
             "sparse_decode_us": att_ms * 1e3,
             "sparse_decode_frac": sb["sparse_decode"] / (att_ms * 1e-3) / 1e9 / hbm_peak,
             "score_topk_us": stg[1] / steps * 1e3,
@@ -486,7 +506,8 @@ def main():
     if args.batch:
         base = base.with_(B=args.batch)
     w = base.with_(seed=base.seed + rank)  # independent replica per rank
-    step = Step(w, fused=not args.unfused)
+    inputs = device_inputs(w)
+    step = Step(w, fused=not args.unfused, inputs=inputs, mode=args.mode)
 
     def barrier():
         if world > 1:
@@ -512,11 +533,11 @@ def main():
 
     # dominant stage of the step and its roofline
     sb = stage_bytes(w)
-    names = Step.STAGES
+    names = ("decode_step",) if args.mode == "step" else Step.STAGES
     dom = max(range(len(stage_ms)), key=lambda i: stage_ms[i])
     dom_ms = stage_ms[dom] / args.steps
     kern = {"label_append": "k_label_append", "score_topk": "k_topk",
-            "sparse_decode": "k_attend"}[names[dom]]
+            "sparse_decode": "k_attend", "decode_step": "k_step"}[names[dom]]
     achieved = sb[names[dom]] / (dom_ms * 1e-3) / 1e9
     traffic = profiled_traffic(kern)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -536,7 +557,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "storage": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                       "T": w.T, "r": w.r, "k": w.k, "fused_score_topk": not args.unfused,
+                       "T": w.T, "r": w.r, "k": w.k, "path": args.mode,
+                       "fused_score_topk": not args.unfused,
                        "l2": "flushed between steps (256 MiB write)", "cuda_graph": True,
                        "parallelism": f"replicas x{world}"},
             "stages": stages, "roofline": roofline,
@@ -546,12 +568,26 @@ def main():
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "us_per_step": te.item() / e2e_steps * 1e3}}
     step.release()
-
+    if args.mode == "step":
+        # the same step as separate calls: per-kernel stage times
+        calls = Step(w, fused=not args.unfused, inputs=inputs, mode="calls")
+        ctot, cst = time_device(calls, max(20, args.steps // 5), 3)
+        cn = max(20, args.steps // 5)
+        calls.release()
+        line["calls"] = {"us_per_step": ctot / cn * 1e3,
+                         "stages": {n: {"us": cst[i] / cn * 1e3,
+                                        "gbs": sb[n] / (cst[i] / cn * 1e-3) / 1e9,
+                                        "frac_of_measured_hbm":
+                                            sb[n] / (cst[i] / cn * 1e-3) / 1e9 / hbm_peak}
+                                    for i, n in enumerate(Step.STAGES)}}
     if rank == 0 and world == 1:
-        dn = dense_entry(w, max(20, args.steps // 10), 3, hbm_peak)
+        dn = dense_entry(w, max(20, args.steps // 10), 3, hbm_peak, inputs=inputs)
         line["dense"] = dn
         line["speedup_vs_dense"] = dn["us_per_step"] / line["us_per_step"]
         line["cpu_baseline"] = time_oracle(base, args.cpu_seconds)
+    del inputs
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1:
         if not args.no_sweep:
             line["sweep"] = run_sweep(w.name, hbm_peak)
     if world > 1:

@@ -76,7 +76,8 @@ enum {
   DS_OP_TOPK = 2,
   DS_OP_SPARSE_DECODE = 3,
   DS_OP_DECODE = 4,
-  DS_OP_SCORE_TOPK = 5
+  DS_OP_SCORE_TOPK = 5,
+  DS_OP_DECODE_STEP = 6
 };
 
 /* Device status bits (ds_device_status). */
@@ -164,6 +165,30 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
 ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
                            float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
                            void* ws, size_t ws_bytes, ds_stream_t stream);
+
+/*
+ * ds_decode_step -- one whole token-sparse decode step: the calls above in the
+ * order a decoder makes them, fused into one launch where the sizes allow.
+ *
+ * With append != 0, first the label row of the newest token (t = T-1) is
+ * written, as ds_label_append(K, C, label, dims, T-1, 1) would; then the top-k
+ * selection of ds_score_topk (the same index set, written to idx) and the
+ * attention of ds_sparse_decode over it.  Double Sparsity's decode: the
+ * calibrated channels pick the important tokens (Method details: Core idea,
+ * Key design) and self-attention runs over those tokens only (Abstract).
+ *
+ * One CTA per query head performs the three phases on chip when r is 8, 16,
+ * 32, 64 or 128, k <= 8192 and the head's selection fits one CTA; otherwise
+ * the three calls are issued on `stream`.  idx: [B*Hq, k] int32 (required).
+ * O and lse as for ds_sparse_decode; the attention's summation order may
+ * differ from ds_sparse_decode's (fp32 rounding only).  ws:
+ * ds_workspace_size(DS_OP_DECODE_STEP, dims, T, k) bytes, zero-filled before
+ * first use (0 bytes when fused).  Other arguments as for the calls above.
+ */
+ds_status ds_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
+                         void* label, int32_t* idx, float* O, float* lse, ds_dims dims,
+                         int32_t T, int32_t k, float scale, int32_t append, void* ws,
+                         size_t ws_bytes, ds_stream_t stream);
 
 /*
  * ds_decode -- dense decode attention over all T cached tokens: the operation

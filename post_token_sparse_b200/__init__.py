@@ -4,7 +4,7 @@ Thin Python binding of ``libds.so`` (C ABI in ``include/ds.h``): argument
 marshalling only.  Every step of the decode path runs in the library's CUDA
 kernels; PyTorch supplies device memory and the current stream.  Importing
 this package fails if the compiled library is missing -- there is no CPU or
-PyTorch fallback.  Build it with ``python -m post_token_sparse_b200.build``.
+PyTorch fallback.  Build it with ``python post_token_sparse_b200/build.py``.
 
 Calls mirror the C ABI:
 
@@ -14,6 +14,8 @@ Calls mirror the C ABI:
     score_topk(Q, C, label, idx, T, scores=None)  the two above in one launch
     sparse_decode(Q, K, V, idx, O, T, scale, lse=None, ws=None)
     decode(Q, K, V, O, T, scale, lse=None, ws=None)   dense reference
+    decode_step(Q, K, V, C, label, idx, O, T, scale, append=True, lse=None, ws=None)
+                                                the three steps above, fused
 
 All tensors must be CUDA, contiguous, with the dtypes and shapes of
 ``include/ds.h``; the C library checks sizes and alignment and raises
@@ -30,7 +32,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
-OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK = range(6)
+(OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK,
+ OP_DECODE_STEP) = range(7)
 DEV_BAD_CHANNEL, DEV_BAD_INDEX = 1, 2
 
 
@@ -55,7 +58,7 @@ class Dims(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing; build it with "
-                          "`python -m post_token_sparse_b200.build`")
+                          "`python post_token_sparse_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, u32p = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)
     st = ctypes.c_int
@@ -68,8 +71,13 @@ def _load():
                              ctypes.c_size_t, vp],
         "ds_decode": [vp, vp, vp, vp, vp, Dims, i32, ctypes.c_float, vp, ctypes.c_size_t, vp],
         "ds_device_status": [u32p, i32, vp],
+        "ds_decode_step": [vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, i32,
+                           vp, ctypes.c_size_t, vp],
     }
     for name, args in sig.items():
+        if not hasattr(lib, name):
+            raise ImportError(f"{LIB_PATH} has no {name}: rebuild it with "
+                              "`python post_token_sparse_b200/build.py --force`")
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = st
@@ -192,6 +200,23 @@ def sparse_decode(Q, K, V, idx, O, T: int, scale: float, lse=None, ws=None):
                                  _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"),
                                  dims, T, k, scale, _ptr(ws, None, "ws"), nbytes,
                                  _stream(Q.device)), "ds_sparse_decode")
+
+
+def decode_step(Q, K, V, C, label, idx, O, T: int, scale: float, append: bool = True,
+                lse=None, ws=None):
+    """One decode step: label row of token T-1 (if append), top-k into idx, attention into O."""
+    dims = dims_of(Q, K, C.shape[1])
+    k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_DECODE_STEP, dims, T, k, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_decode_step(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+                               _ptr(V, torch.bfloat16, "V"), _ptr(C, torch.int32, "C"),
+                               _ptr(label, torch.bfloat16, "label"),
+                               _ptr(idx, torch.int32, "idx"), _ptr(O, torch.float32, "O"),
+                               _ptr(lse, torch.float32, "lse"), dims, T, k, scale,
+                               int(bool(append)), _ptr(ws, None, "ws"), nbytes,
+                               _stream(Q.device)), "ds_decode_step")
 
 
 def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):

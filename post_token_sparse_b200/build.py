@@ -1,6 +1,9 @@
 """Build libds.so (sm_100a) in the package directory.
 
-    python -m post_token_sparse_b200.build [--force]
+    python post_token_sparse_b200/build.py [--force]
+
+(Run as a file, not as ``-m post_token_sparse_b200.build``: importing the
+package loads the library this script builds.)
 
 nvcc cross-compiles for sm_100a without a GPU.  The library links the CUDA
 runtime dynamically so that it shares the runtime (and streams) of the host

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "label.cuh"
 #include "score.cuh"
+#include "step.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -136,6 +137,12 @@ ds_status ensure_attrs() {
     acc(topk_attrs<LabelSource<32>>());
     acc(topk_attrs<LabelSource<64>>());
     acc(topk_attrs<LabelSource<128>>());
+    const size_t step_max = 227 * 1024;
+    acc(allow_smem(k_step<8>, step_max));
+    acc(allow_smem(k_step<16>, step_max));
+    acc(allow_smem(k_step<32>, step_max));
+    acc(allow_smem(k_step<64>, step_max));
+    acc(allow_smem(k_step<128>, step_max));
     g_attr_err[dev] = r;
   });
   return g_attr_err[dev] == cudaSuccess ? DS_OK : cuda_fail(g_attr_err[dev]);
@@ -272,6 +279,28 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
   return launched();
 }
 
+// The fused step applies when r has a vector path, the head's selection fits
+// one CTA, k is small enough for its index list to stay in shared memory, and
+// the whole layout fits a CTA's shared memory.  Depends only on the sizes.
+bool step_fused(const ds_dims& d, int T, int k, int* chunk_out, size_t* smem_out) {
+  const int r = d.r;
+  if (!(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) return false;
+  if (k > kStepMaxK) return false;
+  TopkPlan tp;
+  if (!plan_topk(d.B * d.Hq, T, k, &tp) || tp.cs != 1) return false;
+  const size_t smem = StepLayout(tp.chunk, k).bytes();
+  if (smem > 227 * 1024) return false;
+  *chunk_out = tp.chunk;
+  *smem_out = smem;
+  return true;
+}
+
+template <int R>
+ds_status launch_step(const StepParams& sp, int BH, int chunk, size_t smem, cudaStream_t st) {
+  k_step<R><<<BH, kTopkThreads, smem, st>>>(sp, chunk);
+  return launched();
+}
+
 }  // namespace
 
 extern "C" {
@@ -300,6 +329,13 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
       return partial_bytes(BH, plan_splits(BH, k, true));
     case DS_OP_DECODE:
       return partial_bytes(BH, plan_splits(BH, T, false));
+    case DS_OP_DECODE_STEP: {
+      if (k < 1 || k > T) return 0;
+      int chunk;
+      size_t smem;
+      if (step_fused(dims, T, k, &chunk, &smem)) return 0;
+      return partial_bytes(BH, plan_splits(BH, k, true));
+    }
     default:
       return 0;
   }
@@ -481,4 +517,65 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
+}
+
+extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
+                                    void* label, int32_t* idx, float* O, float* lse,
+                                    ds_dims dims, int32_t T, int32_t k, float scale,
+                                    int32_t append, void* ws, size_t ws_bytes,
+                                    ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !C || !label || !idx || !O || !aligned16(Q) || !aligned16(K) ||
+      !aligned16(V) || !aligned16(C) || !aligned16(label) || !aligned16(idx) || !aligned16(O) ||
+      (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
+  int chunk = 0;
+  size_t smem = 0;
+  const bool fused = step_fused(dims, T, k, &chunk, &smem);
+  if (!fused) {
+    s = check_attend_ws(dims, k, true, ws, ws_bytes);
+    if (s != DS_OK) return s;
+    const bool vec = dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 ||
+                     dims.r == 128;
+    if (!vec) return DS_ERR_UNSUPPORTED;  // the fused score+select needs a vector path
+  }
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  if (fused) {
+    StepParams sp;
+    sp.Q = static_cast<const uint16_t*>(Q);
+    sp.K = static_cast<const uint16_t*>(K);
+    sp.V = static_cast<const uint16_t*>(V);
+    sp.C = C;
+    sp.label = static_cast<uint16_t*>(label);
+    sp.idx = idx;
+    sp.O = O;
+    sp.lse = lse;
+    sp.Hq = dims.Hq;
+    sp.Hkv = dims.Hkv;
+    sp.T_cap = dims.T_cap;
+    sp.T = T;
+    sp.k = k;
+    sp.append = append ? 1 : 0;
+    sp.scale_log2 = scale * 1.4426950408889634f;
+    const int BH = dims.B * dims.Hq;
+    switch (dims.r) {
+      case 8: return launch_step<8>(sp, BH, chunk, smem, stream);
+      case 16: return launch_step<16>(sp, BH, chunk, smem, stream);
+      case 32: return launch_step<32>(sp, BH, chunk, smem, stream);
+      case 64: return launch_step<64>(sp, BH, chunk, smem, stream);
+      default: return launch_step<128>(sp, BH, chunk, smem, stream);
+    }
+  }
+  // the same step as three calls
+  if (append) {
+    s = ds_label_append(K, C, label, dims, T - 1, 1, stream);
+    if (s != DS_OK) return s;
+  }
+  s = ds_score_topk(Q, C, label, nullptr, idx, dims, T, k, stream);
+  if (s != DS_OK) return s;
+  return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
 }

@@ -228,6 +228,9 @@ struct LabelSource {
   const uint16_t* label;
   float* scores;  // optional output
   int Hq, T_cap;
+  int over_t = -1;                  // this token's row is taken from over_row,
+  const uint4* over_row = nullptr;  // not from the label cache (a row written
+                                    // by the same kernel)
   static constexpr int kLanes = R / 8;
   static constexpr int kRowsPerInstr = 32 / kLanes;
   static constexpr int kSlots = 4;
@@ -259,10 +262,11 @@ struct LabelSource {
     for (int base = 0; base < n; base += kStep) {
 #pragma unroll
       for (int i = 0; i < kSlots; ++i) {
-        const uint4 x = v[i];
+        uint4 x = v[i];
         const int jn = slot_item(base + kStep, i);
         if (jn < n) v[i] = ldg_stream(lab + (size_t)tok(jn) * kLanes + chunk);
         const int j = slot_item(base, i);
+        if (over_t >= 0 && j < n && tok(j) == over_t) x = over_row[chunk];
         const float s = lane_group_score<R>(x, qs, chunk);  // all lanes take part
         f(j < n && chunk == 0, j, order_key(s), s);
       }
@@ -383,14 +387,14 @@ __device__ __forceinline__ void digit_hist_pass(const Source& src, int bh, int T
              qs);
 }
 
-// grid (CS, BH), cluster (CS, 1, 1).  chunk: tokens per CTA, a multiple of 32.
+// The selection of one head by one CTA of its cluster (cs CTAs, this one of
+// rank `rank`, shared memory `sm` laid out by TopkLayout(chunk, cs)).  The
+// selected indices, ascending, go to dst_g (global, k entries) and/or dst_s
+// (shared memory, k entries); either may be null.
 template <class Source>
-__global__ void __launch_bounds__(kTopkThreads, 3)  // three CTAs per SM: up to 85 registers
-k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
-  extern __shared__ __align__(16) uint32_t sm[];
-  const int cs = gridDim.x;
-  const int rank = blockIdx.x;  // == cluster rank: the cluster spans grid dimension x
-  const int bh = blockIdx.y;
+__device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int cs, int rank,
+                                          int bh, int T, int k, int chunk, int32_t* dst_g,
+                                          int32_t* dst_s) {
   const TopkLayout L(chunk, cs);
   uint32_t* hist = sm;
   uint32_t* misc = sm + L.small;
@@ -597,7 +601,6 @@ k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
   // rank and its first output position.
   uint32_t tie = eq_before;
   uint32_t out = gt_before + min(eq_before, need);
-  int32_t* dst = idx + (size_t)bh * k;
   for (int base = g0; base < g1; base += 32) {
     const int g = base + lane;
     const uint32_t gmask = g < g1 ? gtm[g] : 0u;
@@ -629,12 +632,24 @@ k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
     while (selm) {
       const int b = __ffs(selm) - 1;
       selm &= selm - 1u;
-      if (pos < (uint32_t)k) dst[pos] = c0 + g * 32 + b;
+      if (pos < (uint32_t)k) {
+        if (dst_g) dst_g[pos] = c0 + g * 32 + b;
+        if (dst_s) dst_s[pos] = c0 + g * 32 + b;
+      }
       ++pos;
     }
     tie += __shfl_sync(0xffffffffu, ne_incl, 31);
     out += __shfl_sync(0xffffffffu, n_incl, 31);
   }
+}
+
+// grid (CS, BH), cluster (CS, 1, 1).  chunk: tokens per CTA, a multiple of 32.
+template <class Source>
+__global__ void __launch_bounds__(kTopkThreads, 3)  // three CTAs per SM: up to 85 registers
+k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
+  extern __shared__ __align__(16) uint32_t sm[];
+  topk_body(src, sm, (int)gridDim.x, (int)blockIdx.x, (int)blockIdx.y, T, k, chunk,
+            idx + (size_t)blockIdx.y * k, nullptr);
 }
 
 }  // namespace ds

@@ -1,0 +1,112 @@
+"""ds_decode_step: the whole decode step in one call, against the three-call path and the oracle.
+
+The index set must equal the one the separate calls produce (the same
+selection code and the same fp32 scores); the label row of the newest token
+must be the oracle's; O is checked against the oracle on the GPU's own set
+(1e-2, as for ds_sparse_decode) and against the three-call path's O (the
+summation order of the attention may differ, so only to fp32 rounding).
+"""
+import numpy as np
+import pytest
+import torch
+
+import dsgen
+import oracle
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import post_token_sparse_b200 as ds
+
+CASES = [
+    # (name, B, Hq, Hkv, T, T_cap, r, k)     fused unless noted
+    ("mha-T1-r8", 1, 2, 2, 1, 1, 8, 1),
+    ("mha-T100-r16", 2, 3, 3, 100, 120, 16, 7),
+    ("gqa-T1000-r16", 2, 8, 2, 1000, 1003, 16, 37),
+    ("mha-T4097-r32", 1, 4, 4, 4097, 4100, 32, 300),
+    ("mha-T3000-r64-kT", 1, 2, 2, 3000, 3000, 64, 3000),
+    ("mha-T2500-r128", 1, 2, 2, 2500, 2600, 128, 777),
+    ("mha-T20000-r8", 2, 4, 4, 20000, 20000, 8, 1250),
+    ("mha-T40000-r8-fallback", 1, 2, 2, 40000, 40000, 8, 10000),   # k > 8192
+    ("mha-T300000-r8-fallback", 1, 1, 1, 300000, 300000, 8, 4000),  # needs a cluster
+]
+
+
+def _run(case, append):
+    name, B, Hq, Hkv, T, T_cap, r, k = case
+    w = dsgen.Workload(name, B=B, Hq=Hq, Hkv=Hkv, T=T_cap, r=r, k=k, n_out=min(8, r),
+                       seed=0x5EED + T)
+    inp = gu.Inputs(w, r=r)
+    BH = B * Hq
+    # label cache up to T-1 (or T when the step does not append); row T-1 stale
+    label = torch.zeros((B, Hq, T_cap, r), dtype=torch.bfloat16, device="cuda")
+    n0 = T - 1 if append else T
+    if n0 > 0:
+        ds.label_append(inp.dK, inp.dC, label, 0, n0)
+    label_sep = label.clone()
+    # the three calls
+    if append:
+        ds.label_append(inp.dK, inp.dC, label_sep, T - 1, 1)
+    idx_sep = torch.empty((BH, k), dtype=torch.int32, device="cuda")
+    ds.score_topk(inp.dQ, inp.dC, label_sep, idx_sep, T)
+    O_sep = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+    ds.sparse_decode(inp.dQ, inp.dK, inp.dV, idx_sep, O_sep, T, w.scale)
+    # the fused step
+    idx = torch.full((BH, k), -1, dtype=torch.int32, device="cuda")
+    O = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ds.decode_step(inp.dQ, inp.dK, inp.dV, inp.dC, label, idx, O, T, w.scale, append=append,
+                   lse=lse)
+    torch.cuda.synchronize()
+    return w, inp, T, label, label_sep, idx, idx_sep, O, O_sep, lse
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("append", [True, False])
+def test_decode_step_matches_three_calls_and_oracle(case, append):
+    w, inp, T, label, label_sep, idx, idx_sep, O, O_sep, lse = _run(case, append)
+    assert torch.equal(idx, idx_sep)
+    got_label = gu.host_bits(label)[:, :, :T]
+    assert np.array_equal(got_label, oracle.label(inp.K[:, :, :T], inp.C, w.Hq))
+    assert (O - O_sep).abs().max().item() <= 1e-5
+    I = idx.cpu().numpy().reshape(w.B, w.Hq, w.k)
+    ref_O, ref_L = oracle.attend(inp.Q, inp.K, inp.V, I, w.scale)
+    assert np.abs(O.cpu().numpy() - ref_O).max() <= 1e-2
+    L = lse.cpu().numpy()
+    assert np.all(np.abs(L - ref_L) <= 1e-3 * (1 + np.abs(ref_L)))
+    assert ds.device_status() == 0
+
+
+def test_decode_step_workspace_only_for_the_fallback():
+    d_fused = ds.Dims(8, 32, 32, 128, 4096, 16)
+    assert ds.workspace_size(ds.OP_DECODE_STEP, d_fused, 4096, 256) == 0
+    d_long = ds.Dims(1, 32, 32, 128, 262144, 8)
+    assert ds.workspace_size(ds.OP_DECODE_STEP, d_long, 262144, 16384) > 0
+
+
+@pytest.mark.parametrize("name", ["llama2-7b-B8-H32-T4K", "sweep-B32-H32-T32K-r8-k2048",
+                                  "gqa-B16-Hq64-Hkv8-T16K"])
+def test_decode_step_full_workload_sampled_heads(name):
+    w = dsgen.workload(name)
+    inp = gu.Inputs(w)
+    BH = w.B * w.Hq
+    label = torch.empty((w.B, w.Hq, w.T, w.r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(inp.dK, inp.dC, label, 0, w.T - 1)
+    idx = torch.empty((BH, w.k), dtype=torch.int32, device="cuda")
+    O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    ds.decode_step(inp.dQ, inp.dK, inp.dV, inp.dC, label, idx, O, w.T, w.scale, append=True)
+    torch.cuda.synchronize()
+    I = idx.cpu().numpy().reshape(w.B, w.Hq, w.k)
+    On = O.cpu().numpy()
+    for b, h in gu.sample_heads(w.B, w.Hq, 10, seed=3):
+        g = h // w.G
+        lab = oracle.label_head(inp.K[b, g], inp.C[h])
+        s64 = oracle.score_head(inp.Q[b, h], inp.C[h], lab)
+        sel = I[b, h]
+        assert len(np.unique(sel)) == w.k and np.all(np.diff(sel) > 0)
+        s_k = np.sort(s64)[::-1][w.k - 1]
+        assert np.all(s64[sel] >= s_k - 1e-3 * (abs(s_k) + 1))
+        o, _, _ = oracle.attend_head(inp.Q[b, h], inp.K[b, g], inp.V[b, g], sel, w.scale)
+        assert np.abs(On[b, h] - o).max() <= 1e-2
+    inp.free()
