@@ -68,6 +68,29 @@ def rank_env():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
+# ---------------------------------------------------------------------------
+# replicas: one process per GPU, each with its own seeded batch, no exchange
+
+def replica_workload(base: dsgen.Workload, rank: int) -> dsgen.Workload:
+    """The workload of one rank: the same shapes, its own seed."""
+    return base.with_(seed=base.seed + rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (a device time): the job ends with its slowest rank."""
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_gbs(bytes_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job algorithmic bandwidth: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -505,7 +528,7 @@ def main():
     base = dsgen.workload(args.workload)
     if args.batch:
         base = base.with_(B=args.batch)
-    w = base.with_(seed=base.seed + rank)  # independent replica per rank
+    w = replica_workload(base, rank)
     inputs = device_inputs(w)
     step = Step(w, fused=not args.unfused, inputs=inputs, mode=args.mode)
 
@@ -518,18 +541,13 @@ def main():
     with ClockSampler(local_rank) as clocks:
         total_ms, stage_ms = time_device(step, args.steps, args.warmup)
     barrier()
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_step = t.item() / args.steps
-    value = world * step_bytes(w) / (ms_step * 1e-3) / 1e9
+    ms_step = max_over_ranks(total_ms, world, "cuda") / args.steps
+    value = job_gbs(step_bytes(w), world, ms_step)
 
     e2e_steps = max(10, min(args.steps, 200))
     e2e_ms, h2d, d2h = time_e2e(step, e2e_steps, 5)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_val = world * step_bytes(w) / (te.item() / e2e_steps * 1e-3) / 1e9
+    e2e_step_ms = max_over_ranks(e2e_ms, world, "cuda") / e2e_steps
+    e2e_val = job_gbs(step_bytes(w), world, e2e_step_ms)
 
     # dominant stage of the step and its roofline
     sb = stage_bytes(w)
@@ -566,7 +584,7 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "us_per_step": te.item() / e2e_steps * 1e3}}
+                    "us_per_step": e2e_step_ms * 1e3}}
     step.release()
     if args.mode == "step":
         # the same step as separate calls: per-kernel stage times
