@@ -54,6 +54,7 @@ def _load():
             lib.dsgen_perm_head.argtypes = [u64, i32, i32, p32]
             lib.dsgen_perm_head.restype = None
             lib.dsgen_hh_positions.argtypes = dims + [p32]
+            lib.dsgen_q_calib.argtypes = [u64, i32, i32, i32, i32, i32, p16]
             _lib = lib
     return _lib
 
@@ -100,6 +101,15 @@ def kv_slab(w: Workload, which: str, b: int, g: int) -> np.ndarray:
     sel = {"K": 0, "V": 1}[which]
     if _load().dsgen_kv_slab(*_dims(w), sel, b, g, _p16(out)) != 0:
         raise ValueError("bad slab")
+    return out
+
+
+def q_calib(w: Workload, Nq: int) -> np.ndarray:
+    """Calibration queries Qc [B,Hq,Nq,d] (bf16 bits): Nq extra queries per head,
+    with the same outlier channels as Q, from a stream of their own."""
+    out = np.empty((w.B, w.Hq, Nq, w.d), np.uint16)
+    if _load().dsgen_q_calib(w.seed, w.B, w.Hq, w.d, w.n_out, Nq, _p16(out)) != 0:
+        raise ValueError("bad calibration request")
     return out
 
 

@@ -26,6 +26,8 @@
  *   - K[b,g,t,c] ~ N(0,1), times 6 on the union of the outlier channels of
  *     the query heads that share KV head g (each channel scaled once);
  *   - V ~ N(0,1);
+ *   - calibration queries Qc[b,h,n,c] (n < Nq) drawn like Q from a stream of
+ *     their own (the offline calibration set of the channel selection);
  *   - optionally n_hh heavy-hitter positions per query head h, where the
  *     channels of C_h (the first r entries of pi_h) of K are overwritten with
  *     6*sqrt(r)*q[C_h]/||q[C_h]||_2, so that those tokens score high.
@@ -39,7 +41,7 @@
 
 #define GAMMA 0x9E3779B97F4A7C15ull
 
-enum { TID_Q = 1, TID_K = 2, TID_V = 3, TID_PERM = 4, TID_HH = 5 };
+enum { TID_Q = 1, TID_K = 2, TID_V = 3, TID_PERM = 4, TID_HH = 5, TID_QCAL = 6 };
 
 static inline uint64_t mix64(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -312,6 +314,35 @@ int dsgen_qkv(uint64_t seed, int B, int Hq, int Hkv, int d, int T, int n_out, in
   for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &P);
   for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
   pthread_mutex_destroy(&P.mu);
+  return 0;
+}
+
+/* Calibration queries Qc[B,Hq,Nq,d] as bf16 bits: N(0,1), times 6 on each
+ * head's outlier channels, element ((b*Hq + h)*Nq + n)*d + c of their stream. */
+int dsgen_q_calib(uint64_t seed, int B, int Hq, int d, int n_out, int Nq, uint16_t* out) {
+  if (B < 1 || Hq < 1 || d < 1 || Nq < 1 || n_out < 0 || n_out > d) return -1;
+  uint64_t s = stream_of(seed, TID_QCAL);
+  int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (size_t)d);
+  char* outlier = (char*)malloc((size_t)d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)d * (size_t)Nq);
+  for (int h = 0; h < Hq; ++h) {
+    memset(outlier, 0, (size_t)d);
+    dsgen_perm_head(seed, h, d, perm);
+    for (int i = 0; i < n_out; ++i) outlier[perm[i]] = 1;
+    for (int b = 0; b < B; ++b) {
+      uint64_t base = ((uint64_t)b * Hq + h) * (uint64_t)Nq * (uint64_t)d;
+      normals(s, base, (size_t)Nq * (size_t)d, z);
+      uint16_t* o = out + base;
+      for (int e = 0; e < Nq * d; ++e) {
+        float f = (float)z[e];
+        if (outlier[e % d]) f *= 6.0f;
+        o[e] = f32_to_bf16_rne(f);
+      }
+    }
+  }
+  free(z);
+  free(outlier);
+  free(perm);
   return 0;
 }
 

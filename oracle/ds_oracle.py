@@ -38,6 +38,17 @@ float64 on the exact decoded values.  ``s32`` (float64 scores rounded to
 float32, nearest-even) is what the bit-exact top-k parity check feeds to the
 GPU top-k.
 
+Offline channel calibration (the step before the path).  The page says the
+channel pattern is static, so it is fixed offline (Method details: Core idea;
+Technical framework), and leaves the criterion open (Key design: "unknown").
+The reading taken here, the plainest one:
+
+  importance  I[h,c] = mean over the pairs (calibration query n, cached token t)
+              of the same sequence b of |q[b,h,n,c] * k[b,g(h),t,c]|, the
+              magnitude of channel c's share of the attention logit
+  selection   the r channels with the largest I[h,c]; ties go to the lower
+              channel; output ascending
+
 Pins (see tests/test_oracle_pins.py): bf16 decoding against known bit
 patterns; label gather against the identity/permutation cases and a
 per-element brute force; score against one-hot queries and the attention
@@ -58,6 +69,7 @@ __all__ = [
     "bf16_to_f64", "label_head", "label", "score_head", "score", "to_f32",
     "topk_head", "topk", "attend_head", "attend", "dense", "lse_merge",
     "attend_split_head", "sparse_step", "group_of",
+    "calibrate_importance", "calibrate_select", "calibrate",
 ]
 
 
@@ -237,3 +249,40 @@ def sparse_step(Q, K, V, C, k, scale):
     idx = topk(s32, k)
     O, L = attend(Q, K, V, idx, scale)
     return {"label": lab, "s64": s64, "s32": s32, "idx": idx, "O": O, "lse": L}
+
+
+# ---- offline channel calibration -------------------------------------------------
+
+def calibrate_importance(Qc: np.ndarray, K: np.ndarray, T: int, Hq: int) -> np.ndarray:
+    """I[h, c] = 1/(B*Nq*T) * sum_b sum_n sum_t |q[b,h,n,c] * k[b,g(h),t,c]|.
+
+    Qc [B,Hq,Nq,d] calibration queries and K [B,Hkv,T_cap,d] keys (bf16 bits);
+    tokens 0..T-1.  |q k| = |q| |k|, so for each sequence b the double sum over
+    (n, t) is the product of the two single sums.  Returns [Hq, d] float64.
+    """
+    B, _, Nq, d = Qc.shape
+    Hkv = K.shape[1]
+    I = np.zeros((Hq, d))
+    for b in range(B):
+        ksum = [np.abs(bf16_to_f64(K[b, g, :T])).sum(axis=0) for g in range(Hkv)]
+        for h in range(Hq):
+            qsum = np.abs(bf16_to_f64(Qc[b, h])).sum(axis=0)
+            I[h] += qsum * ksum[group_of(h, Hq, Hkv)]
+    return I / (B * Nq * T)
+
+
+def calibrate_select(I: np.ndarray, r: int) -> np.ndarray:
+    """C [Hq, r]: per head the r channels of largest importance, ties to the
+    lower channel, in ascending channel order."""
+    Hq, d = I.shape
+    C = np.empty((Hq, r), np.int32)
+    for h in range(Hq):
+        order = np.lexsort((np.arange(d), -np.asarray(I[h], np.float64)))
+        C[h] = np.sort(order[:r])
+    return C
+
+
+def calibrate(Qc: np.ndarray, K: np.ndarray, T: int, Hq: int, r: int):
+    """(C [Hq, r] int32, I [Hq, d] float64) for a calibration set."""
+    I = calibrate_importance(Qc, K, T, Hq)
+    return calibrate_select(I, r), I

@@ -20,6 +20,10 @@ What pins what:
                       torch.logsumexp for the LSE; the worked example
   merge               split invariance against the unsplit result
   whole step          r = d, k = T equals dense attention
+  calibration         brute-force mean over (query, token) pairs; the
+                      query-head -> KV-head map on marked KV heads; ties to
+                      the lower channel; channel-permutation equivariance;
+                      recovery of the generator's seeded outlier channels
 """
 from __future__ import annotations
 
@@ -307,5 +311,83 @@ def pin_f32_rounding(orc):
     assert np.isinf(got[3])
 
 
+# ---------------------------------------------------------------------------
+# offline channel calibration
+
+def pin_calib_bruteforce(orc):
+    rng = np.random.default_rng(41)
+    B, Hq, Hkv, Nq, T, Tcap, d = 2, 4, 2, 3, 5, 7, 8
+    Qc = _rand_bits(rng, (B, Hq, Nq, d), 2.0)
+    K = _rand_bits(rng, (B, Hkv, Tcap, d), 1.5)
+    I = orc.calibrate_importance(Qc, K, T, Hq)
+    qf, kf = _f(Qc), _f(K)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        for c in range(d):
+            tot = 0.0
+            for b in range(B):
+                for n in range(Nq):
+                    for t in range(T):
+                        tot += abs(qf[b, h, n, c] * kf[b, g, t, c])
+            ref = tot / (B * Nq * T)
+            assert abs(I[h, c] - ref) <= 1e-12 * (1 + ref), (h, c, I[h, c], ref)
+
+
+def pin_calib_groups_and_order(orc):
+    # KV head g is large only on channel 5 + g: query head h picks 5 + g(h)
+    B, Hq, Hkv, Nq, T, d = 1, 6, 3, 2, 4, 16
+    Qc = _bits(np.ones((B, Hq, Nq, d)))
+    K = np.empty((B, Hkv, T, d), np.uint16)
+    for g in range(Hkv):
+        x = np.full((T, d), 0.5)
+        x[:, 5 + g] = -4.0  # magnitude counts, not sign
+        K[0, g] = _bits(x)
+    C, I = orc.calibrate(Qc, K, T, Hq, 1)
+    for h in range(Hq):
+        assert C[h, 0] == 5 + h // 2, (h, C[h])
+        assert I[h, 5 + h // 2] == 4.0 and I[h, 0] == 0.5
+    # r = 3: the large channel plus ties at 0.5 broken toward the lowest channels
+    C3, _ = orc.calibrate(Qc, K, T, Hq, 3)
+    for h in range(Hq):
+        assert list(C3[h]) == [0, 1, 5 + h // 2], (h, C3[h])
+    # all equal: channels 0..r-1, ascending
+    Ce, _ = orc.calibrate(Qc, _bits(np.ones((B, Hkv, T, d))), T, Hq, 4)
+    assert np.array_equal(Ce, np.tile(np.arange(4, dtype=np.int32), (Hq, 1)))
+    # explicit selection order: descending importance, ascending output
+    Isel = np.array([[0.1, 3.0, 2.0, 3.0, -1.0, 2.5]])
+    assert list(orc.calibrate_select(Isel, 3)[0]) == [1, 3, 5]
+    assert list(orc.calibrate_select(Isel, 4)[0]) == [1, 2, 3, 5]
+
+
+def pin_calib_permutation(orc):
+    rng = np.random.default_rng(43)
+    B, Hq, Hkv, Nq, T, d = 2, 2, 1, 4, 9, 12
+    Qc = _rand_bits(rng, (B, Hq, Nq, d))
+    K = _rand_bits(rng, (B, Hkv, T, d))
+    perm = rng.permutation(d)
+    I = orc.calibrate_importance(Qc, K, T, Hq)
+    Ip = orc.calibrate_importance(Qc[..., perm], K[..., perm], T, Hq)
+    assert np.allclose(Ip, I[:, perm], rtol=1e-13, atol=0)
+    # tokens past T are ignored
+    K2 = K.copy()
+    K2[:, :, T - 1] = _bits(np.full(d, 100.0))
+    assert not np.allclose(orc.calibrate_importance(Qc, K2, T, Hq), I)
+    assert np.allclose(orc.calibrate_importance(Qc, K2, T - 1, Hq),
+                       orc.calibrate_importance(Qc, K, T - 1, Hq))
+
+
+def pin_calib_recovers_outliers(orc):
+    # generator property: Q and K are scaled x6 on each head's n_out outlier
+    # channels, so those channels carry the largest |q_c k_c|
+    w = dsgen.Workload("calib-pin", B=2, Hq=4, Hkv=2, T=256, r=8, k=16, n_out=8, seed=0xCA11)
+    _, K, _ = dsgen.qkv(w, want=("K",))
+    Qc = dsgen.q_calib(w, 16)
+    C, _ = orc.calibrate(Qc, K, w.T, w.Hq, w.n_out)
+    for h in range(w.Hq):
+        assert np.array_equal(C[h], dsgen.outliers(w, h)), (h, C[h], dsgen.outliers(w, h))
+
+
 PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
-        pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding]
+        pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding,
+        pin_calib_bruteforce, pin_calib_groups_and_order, pin_calib_permutation,
+        pin_calib_recovers_outliers]

@@ -49,6 +49,23 @@ MUTATIONS = [
     ("dense drops last token", "idx = np.broadcast_to(np.arange(T, dtype=np.int32), (B, Hq, T))",
      "idx = np.broadcast_to(np.arange(T - 1, dtype=np.int32), (B, Hq, T - 1))"),
     ("step selects on float64 scores with wrong k", "idx = topk(s32, k)", "idx = topk(s32, max(1, k - 1))"),
+    ("calibration without magnitudes", "qsum = np.abs(bf16_to_f64(Qc[b, h])).sum(axis=0)",
+     "qsum = bf16_to_f64(Qc[b, h]).sum(axis=0)"),
+    ("calibration keys without magnitudes", "ksum = [np.abs(bf16_to_f64(K[b, g, :T])).sum(axis=0)",
+     "ksum = [bf16_to_f64(K[b, g, :T]).sum(axis=0)"),
+    ("calibration reads past T", "ksum = [np.abs(bf16_to_f64(K[b, g, :T])).sum(axis=0)",
+     "ksum = [np.abs(bf16_to_f64(K[b, g])).sum(axis=0)"),
+    ("calibration sums q and k instead of the product", "I[h] += qsum * ksum[group_of(h, Hq, Hkv)]",
+     "I[h] += qsum + ksum[group_of(h, Hq, Hkv)]"),
+    ("calibration pairs the wrong KV head", "I[h] += qsum * ksum[group_of(h, Hq, Hkv)]",
+     "I[h] += qsum * ksum[h % Hkv]"),
+    ("calibration mean over the wrong count", "return I / (B * Nq * T)", "return I / (Nq * T)"),
+    ("calibration picks the smallest", "order = np.lexsort((np.arange(d), -np.asarray(I[h], np.float64)))",
+     "order = np.lexsort((np.arange(d), np.asarray(I[h], np.float64)))"),
+    ("calibration ties to the higher channel",
+     "order = np.lexsort((np.arange(d), -np.asarray(I[h], np.float64)))",
+     "order = np.lexsort((-np.arange(d), -np.asarray(I[h], np.float64)))"),
+    ("calibration output unsorted", "C[h] = np.sort(order[:r])", "C[h] = order[:r]"),
 ]
 
 
