@@ -49,6 +49,17 @@ The reading taken here, the plainest one:
   selection   the r channels with the largest I[h,c]; ties go to the lower
               channel; output ascending
 
+Group-shared selection (grouped KV heads).  The page's token sparsity keeps
+the important tokens of the attention (Abstract; Key points 2); with grouped
+KV heads the G query heads of a group read the same K/V rows, so one
+selection per group lets each row be read once for all of them.  The page
+does not define a group score; the reading taken here:
+
+  group score  sg[b,g,t] = sum over the query heads h of group g of s[b,h,t]
+               (the per-head approximate scores; head order h = gG .. gG+G-1)
+  group top-k  the k tokens of largest sg, with the per-head top-k's order
+  attention    every query head of the group attends over the group's set
+
 Pins (see tests/test_oracle_pins.py): bf16 decoding against known bit
 patterns; label gather against the identity/permutation cases and a
 per-element brute force; score against one-hot queries and the attention
@@ -70,6 +81,7 @@ __all__ = [
     "topk_head", "topk", "attend_head", "attend", "dense", "lse_merge",
     "attend_split_head", "sparse_step", "group_of",
     "calibrate_importance", "calibrate_select", "calibrate",
+    "group_score", "group_attend", "group_sparse_step",
 ]
 
 
@@ -286,3 +298,44 @@ def calibrate(Qc: np.ndarray, K: np.ndarray, T: int, Hq: int, r: int):
     """(C [Hq, r] int32, I [Hq, d] float64) for a calibration set."""
     I = calibrate_importance(Qc, K, T, Hq)
     return calibrate_select(I, r), I
+
+
+# ---- group-shared selection ------------------------------------------------------
+
+def group_score(s: np.ndarray, Hkv: int) -> np.ndarray:
+    """sg [B, Hkv, T]: the sum of the per-head scores s [B, Hq, T] over the
+    query heads of each KV group, added in head order."""
+    B, Hq, T = s.shape
+    G = Hq // Hkv
+    sg = np.zeros((B, Hkv, T), dtype=s.dtype)
+    for h in range(Hq):
+        sg[:, group_of(h, Hq, Hkv)] += s[:, h]
+    return sg
+
+
+def group_attend(Q, K, V, idx_g, scale):
+    """O [B, Hq, d], lse [B, Hq]: query head h attends over its group's set
+    idx_g [B, Hkv, k]."""
+    B, Hq, _ = Q.shape
+    Hkv = K.shape[1]
+    idx = np.empty((B, Hq, idx_g.shape[-1]), np.int32)
+    for h in range(Hq):
+        idx[:, h] = idx_g[:, group_of(h, Hq, Hkv)]
+    return attend(Q, K, V, idx, scale)
+
+
+def group_sparse_step(Q, K, V, C, k, scale):
+    """label -> per-head scores -> group scores -> group top-k -> attention.
+
+    The group scores are summed from the float32-rounded per-head scores in
+    float32 (sg32, what a float32 pipeline selects on) and in float64 (sg64).
+    """
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    lab = label(K, C, Hq)
+    s64 = score(Q, C, lab)
+    s32 = to_f32(s64)
+    sg64 = group_score(s64, Hkv)
+    sg32 = group_score(s32.astype(np.float32), Hkv)
+    idx = topk(sg32, k)
+    O, L = group_attend(Q, K, V, idx, scale)
+    return {"label": lab, "s64": s64, "sg64": sg64, "sg32": sg32, "idx": idx, "O": O, "lse": L}

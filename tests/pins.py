@@ -20,6 +20,10 @@ What pins what:
                       torch.logsumexp for the LSE; the worked example
   merge               split invariance against the unsplit result
   whole step          r = d, k = T equals dense attention
+  group selection     brute-force sums over the heads of each group; one
+                      head per group is the per-head path; identical heads
+                      keep the per-head set; group attention equals per-head
+                      attention on the broadcast set
   calibration         brute-force mean over (query, token) pairs; the
                       query-head -> KV-head map on marked KV heads; ties to
                       the lower channel; channel-permutation equivariance;
@@ -387,7 +391,68 @@ def pin_calib_recovers_outliers(orc):
         assert np.array_equal(C[h], dsgen.outliers(w, h)), (h, C[h], dsgen.outliers(w, h))
 
 
+# ---------------------------------------------------------------------------
+# group-shared selection
+
+def pin_group_score(orc):
+    rng = np.random.default_rng(51)
+    B, Hq, Hkv, T = 2, 6, 2, 7
+    s = rng.standard_normal((B, Hq, T))
+    sg = orc.group_score(s, Hkv)
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(T):
+                ref = s[b, 3 * g, t] + s[b, 3 * g + 1, t] + s[b, 3 * g + 2, t]
+                assert sg[b, g, t] == ref  # same addition order, exact
+    # float32 input is summed in float32 (round after each addition)
+    s32 = np.array([[[1.0], [2.0 ** -24], [2.0 ** -24]]], np.float32)
+    assert orc.group_score(s32, 1)[0, 0, 0] == np.float32(1.0)
+    # one head per group: the per-head scores unchanged
+    assert np.array_equal(orc.group_score(s, Hq), s)
+
+
+def pin_group_step(orc):
+    rng = np.random.default_rng(52)
+    B, Hkv, G, T, d, r, k = 1, 2, 3, 40, 16, 4, 6
+    Hq = Hkv * G
+    Q = _rand_bits(rng, (B, Hq, d))
+    K = _rand_bits(rng, (B, Hkv, T, d))
+    V = _rand_bits(rng, (B, Hkv, T, d))
+    C = np.sort(np.stack([rng.permutation(d)[:r] for _ in range(Hq)]), axis=1).astype(np.int32)
+    scale = 0.25
+    res = orc.group_sparse_step(Q, K, V, C, k, scale)
+    # brute force: group scores from explicit dot products, then a full sort
+    qf, kf = _f(Q), _f(K)
+    for g in range(Hkv):
+        sg = [sum(sum(qf[0, h, c] * kf[0, g, t, c] for c in C[h]) for h in range(g * G, g * G + G))
+              for t in range(T)]
+        assert np.allclose(res["sg64"][0, g], sg, rtol=1e-12, atol=1e-12)
+        order = sorted(range(T), key=lambda t: (-float(res["sg32"][0, g, t]), t))[:k]
+        assert list(res["idx"][0, g]) == sorted(order)
+        # every head of the group attends over the group's set
+        for h in range(g * G, g * G + G):
+            o, lse, _ = orc.attend_head(Q[0, h], K[0, g], V[0, g], res["idx"][0, g], scale)
+            assert np.allclose(res["O"][0, h], o) and abs(res["lse"][0, h] - lse) < 1e-12
+    # one query head per KV head: the per-head step
+    Q1, C1 = Q[:, :Hkv], C[:Hkv]
+    one = orc.group_sparse_step(Q1, K, V, C1, k, scale)
+    per = orc.sparse_step(Q1, K, V, C1, k, scale)
+    assert np.array_equal(one["idx"], per["idx"]) and np.allclose(one["O"], per["O"])
+    # G identical heads: the group keeps the single head's set
+    Qr = np.repeat(Q1, G, axis=1)
+    Cr = np.repeat(C1, G, axis=0)
+    rep = orc.group_sparse_step(Qr, K, V, Cr, k, scale)
+    sg64 = rep["sg64"]
+    for g in range(Hkv):
+        want = sorted(sorted(range(T), key=lambda t: (-per["s64"][0, g, t], t))[:k])
+        got = list(rep["idx"][0, g])
+        # equal up to float32 near-ties of the single head's scores
+        if got != want:
+            kth = np.sort(sg64[0, g])[::-1][k - 1]
+            assert all(sg64[0, g, t] >= kth - 1e-6 * (abs(kth) + 1) for t in got)
+
+
 PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
         pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding,
         pin_calib_bruteforce, pin_calib_groups_and_order, pin_calib_permutation,
-        pin_calib_recovers_outliers]
+        pin_calib_recovers_outliers, pin_group_score, pin_group_step]

@@ -66,6 +66,16 @@ MUTATIONS = [
      "order = np.lexsort((np.arange(d), -np.asarray(I[h], np.float64)))",
      "order = np.lexsort((-np.arange(d), -np.asarray(I[h], np.float64)))"),
     ("calibration output unsorted", "C[h] = np.sort(order[:r])", "C[h] = order[:r]"),
+    ("group score takes the wrong group", "sg[:, group_of(h, Hq, Hkv)] += s[:, h]",
+     "sg[:, h % Hkv] += s[:, h]"),
+    ("group score keeps the last head only", "sg[:, group_of(h, Hq, Hkv)] += s[:, h]",
+     "sg[:, group_of(h, Hq, Hkv)] = s[:, h]"),
+    ("group score in float64 for the float32 pipeline",
+     "sg = np.zeros((B, Hkv, T), dtype=s.dtype)", "sg = np.zeros((B, Hkv, T))"),
+    ("group attention uses the first group's set", "idx[:, h] = idx_g[:, group_of(h, Hq, Hkv)]",
+     "idx[:, h] = idx_g[:, 0]"),
+    ("group step selects on the first heads' own scores", "idx = topk(sg32, k)",
+     "idx = topk(s32[:, :Hkv], k)"),
 ]
 
 
