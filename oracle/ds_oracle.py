@@ -60,6 +60,21 @@ does not define a group score; the reading taken here:
   group top-k  the k tokens of largest sg, with the per-head top-k's order
   attention    every query head of the group attends over the group's set
 
+Block-granular selection (page "Jenga: Enhancing LLM Long-Context Fine-tuning
+with Contextual Token Sparsity", Core method 1: Information-driven Token
+Elimination; Observation 2 gives the default block of 64 tokens).  There a
+token's informativeness sums only the positive attention scores it receives,
+a block's informativeness is the largest of its tokens', and blocks are kept
+against a threshold tuned per layer on a model.  For one decode query, with no
+model to tune a threshold on, the reading taken is:
+
+  token        I[t] = max(s[t], 0) (s the approximate score above)
+  block        Ib[j] = max over t in [j*bs, min((j+1)*bs, T)) of I[t]
+  selection    a fixed count: the kb blocks of largest Ib, ties to the lower
+               block (the decode analogue of the top-k above); the kept tokens
+               are every token of those blocks (clipped to T), ascending
+  attention    as above, over the kept tokens
+
 Pins (see tests/test_oracle_pins.py): bf16 decoding against known bit
 patterns; label gather against the identity/permutation cases and a
 per-element brute force; score against one-hot queries and the attention
@@ -82,6 +97,7 @@ __all__ = [
     "attend_split_head", "sparse_step", "group_of",
     "calibrate_importance", "calibrate_select", "calibrate",
     "group_score", "group_attend", "group_sparse_step",
+    "block_score", "block_tokens", "block_sparse_step",
 ]
 
 
@@ -339,3 +355,44 @@ def group_sparse_step(Q, K, V, C, k, scale):
     idx = topk(sg32, k)
     O, L = group_attend(Q, K, V, idx, scale)
     return {"label": lab, "s64": s64, "sg64": sg64, "sg32": sg32, "idx": idx, "O": O, "lse": L}
+
+
+# ---- block-granular selection ----------------------------------------------------
+
+def block_score(s: np.ndarray, bs: int) -> np.ndarray:
+    """Ib [..., ceil(T/bs)]: per block of bs consecutive tokens, the largest
+    positive part max(s_t, 0) of its tokens' scores (the last block may be short)."""
+    s = np.asarray(s)
+    T = s.shape[-1]
+    nb = -(-T // bs)
+    out = np.empty(s.shape[:-1] + (nb,), dtype=s.dtype)
+    for j in range(nb):
+        out[..., j] = np.maximum(s[..., j * bs:min((j + 1) * bs, T)], 0).max(axis=-1)
+    return out
+
+
+def block_tokens(bidx: np.ndarray, bs: int, T: int) -> np.ndarray:
+    """Ascending token indices of the blocks ``bidx`` (one head), clipped to T."""
+    toks = [t for j in sorted(int(x) for x in bidx) for t in range(j * bs, min((j + 1) * bs, T))]
+    return np.asarray(toks, dtype=np.int32)
+
+
+def block_sparse_step(Q, K, V, C, bs, kb, scale):
+    """label -> scores -> block scores (on the float32-rounded scores) -> top-kb
+    blocks -> attention of each head over its blocks' tokens."""
+    B, Hq, _ = Q.shape
+    Hkv = K.shape[1]
+    T = K.shape[2]
+    lab = label(K, C, Hq)
+    s64 = score(Q, C, lab)
+    s32 = to_f32(s64)
+    sb = block_score(s32, bs)
+    bidx = topk(sb, kb)
+    O = np.empty((B, Hq, Q.shape[2]))
+    L = np.empty((B, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            g = group_of(h, Hq, Hkv)
+            toks = block_tokens(bidx[b, h], bs, T)
+            O[b, h], L[b, h], _ = attend_head(Q[b, h], K[b, g], V[b, g], toks, scale)
+    return {"s32": s32, "sb": sb, "bidx": bidx, "O": O, "lse": L}

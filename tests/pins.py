@@ -24,6 +24,10 @@ What pins what:
                       head per group is the per-head path; identical heads
                       keep the per-head set; group attention equals per-head
                       attention on the broadcast set
+  block selection     brute-force block maxima of the positive parts, short
+                      last block; bs = 1 is top-k of the clamped scores;
+                      blocks' tokens contiguous and clipped; the step equals
+                      attention over the blocks' tokens
   calibration         brute-force mean over (query, token) pairs; the
                       query-head -> KV-head map on marked KV heads; ties to
                       the lower channel; channel-permutation equivariance;
@@ -452,7 +456,53 @@ def pin_group_step(orc):
             assert all(sg64[0, g, t] >= kth - 1e-6 * (abs(kth) + 1) for t in got)
 
 
+# ---------------------------------------------------------------------------
+# block-granular selection
+
+def pin_block_score(orc):
+    s = np.array([[-1.0, 3.0, -2.0, 0.5, -0.25, -4.0, 7.0, -1.0, 2.0, -3.0]])
+    # bs = 4: blocks [-1,3,-2,.5] [-.25,-4,7,-1] [2,-3] (short); negative-only block -> 0
+    assert np.array_equal(orc.block_score(s, 4), [[3.0, 7.0, 2.0]])
+    assert np.array_equal(orc.block_score(np.array([[-1.0, -2.0, -0.5]]), 2), [[0.0, 0.0]])
+    rng = np.random.default_rng(61)
+    x = rng.standard_normal((3, 37))
+    for bs in (1, 2, 5, 8, 37, 64):
+        got = orc.block_score(x, bs)
+        for i in range(3):
+            ref = [max(0.0, max(x[i, j:j + bs])) for j in range(0, 37, bs)]
+            assert list(got[i]) == ref, (bs, i)
+    # bs = 1: the positive-clamped scores themselves
+    assert np.array_equal(orc.block_score(x, 1), np.maximum(x, 0))
+
+
+def pin_block_tokens_and_step(orc):
+    assert list(orc.block_tokens(np.array([2, 0]), 4, 10)) == [0, 1, 2, 3, 8, 9]
+    assert list(orc.block_tokens(np.array([1]), 3, 5)) == [3, 4]
+    rng = np.random.default_rng(62)
+    B, Hq, Hkv, T, d, r = 1, 2, 1, 50, 16, 4
+    Q = _rand_bits(rng, (B, Hq, d))
+    K = _rand_bits(rng, (B, Hkv, T, d))
+    V = _rand_bits(rng, (B, Hkv, T, d))
+    C = np.sort(np.stack([rng.permutation(d)[:r] for _ in range(Hq)]), axis=1).astype(np.int32)
+    scale = 0.3
+    bs, kb = 8, 3
+    res = orc.block_sparse_step(Q, K, V, C, bs, kb, scale)
+    qf, kf = _f(Q), _f(K)
+    for h in range(Hq):
+        s = [np.float32(sum(qf[0, h, c] * kf[0, 0, t, c] for c in C[h])) for t in range(T)]
+        blocks = [max(0.0, max(float(v) for v in s[j:j + bs])) for j in range(0, T, bs)]
+        order = sorted(range(len(blocks)), key=lambda j: (-blocks[j], j))[:kb]
+        assert list(res["bidx"][0, h]) == sorted(order)
+        toks = [t for j in sorted(order) for t in range(j * bs, min(j * bs + bs, T))]
+        o, lse, _ = orc.attend_head(Q[0, h], K[0, 0], V[0, 0], np.array(toks), scale)
+        assert np.allclose(res["O"][0, h], o) and abs(res["lse"][0, h] - lse) < 1e-12
+    # bs = 1 selects the top-k of the positive-clamped float32 scores
+    one = orc.block_sparse_step(Q, K, V, C, 1, 5, scale)
+    assert np.array_equal(one["bidx"], orc.topk(np.maximum(one["s32"], 0), 5))
+
+
 PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
         pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding,
         pin_calib_bruteforce, pin_calib_groups_and_order, pin_calib_permutation,
-        pin_calib_recovers_outliers, pin_group_score, pin_group_step]
+        pin_calib_recovers_outliers, pin_group_score, pin_group_step, pin_block_score,
+        pin_block_tokens_and_step]

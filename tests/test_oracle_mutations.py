@@ -76,6 +76,18 @@ MUTATIONS = [
      "idx[:, h] = idx_g[:, 0]"),
     ("group step selects on the first heads' own scores", "idx = topk(sg32, k)",
      "idx = topk(s32[:, :Hkv], k)"),
+    ("block score keeps negative scores",
+     "out[..., j] = np.maximum(s[..., j * bs:min((j + 1) * bs, T)], 0).max(axis=-1)",
+     "out[..., j] = s[..., j * bs:min((j + 1) * bs, T)].max(axis=-1)"),
+    ("block score sums instead of max",
+     "out[..., j] = np.maximum(s[..., j * bs:min((j + 1) * bs, T)], 0).max(axis=-1)",
+     "out[..., j] = np.maximum(s[..., j * bs:min((j + 1) * bs, T)], 0).sum(axis=-1)"),
+    ("block score drops the short last block", "nb = -(-T // bs)", "nb = T // bs"),
+    ("block tokens off by one", "for t in range(j * bs, min((j + 1) * bs, T))]",
+     "for t in range(j * bs + 1, min((j + 1) * bs + 1, T))]"),
+    ("block tokens not clipped", "for t in range(j * bs, min((j + 1) * bs, T))]",
+     "for t in range((j * bs), (j + 1) * bs)]"),
+    ("block step selects on tokens, not blocks", "bidx = topk(sb, kb)", "bidx = topk(s32, kb)"),
 ]
 
 
