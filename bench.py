@@ -383,15 +383,12 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
     C = dsgen.channels(w)
     per_head = w.T * w.r * 2 + w.k * 4 * w.d + w.d * 6
     done, elapsed, dense_el = 0, 0.0, 0.0
-    for p in order:
-        b, h = divmod(int(p), w.Hq)
-        g = h // w.G
-        q = dsgen.q_slab(w, b, h)
-        Kbg = dsgen.kv_slab(w, "K", b, g)
-        Vbg = dsgen.kv_slab(w, "V", b, g)
-        lab = oracle.label_head(Kbg, C[h])  # label cache: setup, not timed
+    cache, cached_bytes, passes = [], 0, 0
+
+    def run_head(q, Ch, lab, Kbg, Vbg):
+        nonlocal elapsed, dense_el
         t0 = time.perf_counter()
-        s = oracle.to_f32(oracle.score_head(q, C[h], lab))
+        s = oracle.to_f32(oracle.score_head(q, Ch, lab))
         idx = oracle.topk_head(s, w.k)
         oracle.attend_head(q, Kbg, Vbg, idx, w.scale)
         elapsed += time.perf_counter() - t0
@@ -399,16 +396,36 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
             t0 = time.perf_counter()
             oracle.attend_head(q, Kbg, Vbg, np.arange(w.T), w.scale)
             dense_el += time.perf_counter() - t0
+
+    for p in order:
+        b, h = divmod(int(p), w.Hq)
+        g = h // w.G
+        q = dsgen.q_slab(w, b, h)
+        Kbg = dsgen.kv_slab(w, "K", b, g)
+        Vbg = dsgen.kv_slab(w, "V", b, g)
+        lab = oracle.label_head(Kbg, C[h])  # label cache: setup, not timed
+        run_head(q, C[h], lab, Kbg, Vbg)
         done += 1
+        if cached_bytes <= (2 << 30):  # keep the inputs for further passes
+            cache.append((q, C[h], lab, Kbg, Vbg))
+            cached_bytes += Kbg.nbytes + Vbg.nbytes + lab.nbytes
         if elapsed + dense_el >= budget_s:
             break
+    passes = 1
+    # a short workload is timed over repeated passes (inputs kept), up to the budget
+    while len(cache) == w.B * w.Hq and elapsed + dense_el < budget_s and passes < 1000:
+        for item in cache:
+            run_head(*item)
+            done += 1
+        passes += 1
     if limit is not None:
         limit.unregister() if hasattr(limit, "unregister") else None
     us_step = elapsed / done * w.B * w.Hq * 1e6
     out = {"value": per_head * done / elapsed / 1e9, "unit": "GB/s", "cores": 1,
            "kind": "oracle", "us_per_step": us_step,
-           "sample": f"{done} of {w.B * w.Hq} heads of {w.name}, score + top-k + attention "
-                     f"per head in float64 numpy, one thread ({elapsed:.1f} s)"}
+           "sample": f"{done} head-steps ({passes} pass(es) over the {w.B * w.Hq} heads) of "
+                     f"{w.name}, score + top-k + attention per head in float64 numpy, one "
+                     f"thread ({elapsed:.1f} s)"}
     if with_dense:
         out["dense_us_per_step"] = dense_el / done * w.B * w.Hq * 1e6
     return out
@@ -452,6 +469,9 @@ def sweep_entry(w, steps, warmup, hbm_peak, fused=True, inputs=None):
     sc = Step(w, fused=fused, inputs=inputs, mode="calls")
     _, stg = time_device(sc, steps, warmup)
     sc.release()
+    su = Step(w, fused=False, inputs=inputs, mode="calls")  # score, then top-k over the scores
+    _, stu = time_device(su, steps, warmup)
+    su.release()
     sb = stage_bytes(w)
     att_ms = stg[2] / steps
     return {"us_per_step": ms * 1e3, "gbs": step_bytes(w) / (ms * 1e-3) / 1e9,
@@ -461,6 +481,7 @@ def sweep_entry(w, steps, warmup, hbm_peak, fused=True, inputs=None):
             "sparse_decode_frac": sb["sparse_decode"] / (att_ms * 1e-3) / 1e9 / hbm_peak,
             "score_topk_us": stg[1] / steps * 1e3,
             "score_topk_frac": sb["score_topk"] / (stg[1] / steps * 1e-3) / 1e9 / hbm_peak,
+            "score_then_topk_us": stu[1] / steps * 1e3,
             "tokens_heads_per_s": w.B * w.Hq * w.T / (ms * 1e-3)}
 
 
@@ -471,6 +492,118 @@ def dense_entry(w, steps, warmup, hbm_peak, inputs=None):
     ms = tot / steps
     return {"us_per_step": ms * 1e3, "gbs": w.dense_bytes() / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": w.dense_bytes() / (ms * 1e-3) / 1e9 / hbm_peak}
+
+
+def time_graph(fn, steps: int, warmup: int) -> float:
+    """Mean device ms of fn() (a few launches) replayed as a CUDA graph, with the
+    L2 flushed (256 MiB write) before each replay."""
+    import torch
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    fn()  # eager once: one-time setup outside the capture
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        e0.record()
+        fn()
+        e1.record()
+    for _ in range(warmup):
+        flush.zero_()
+        g.replay()
+    tot = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    del g
+    return tot / steps
+
+
+def calib_entry(w, K, hbm_peak, nq: int = 16, steps: int = 50):
+    """Offline channel calibration (ds_calibrate) over the workload's keys and nq
+    calibration queries per head: reads K once and the queries once."""
+    import numpy as np
+    import torch
+
+    import post_token_sparse_b200 as ds
+
+    qc = dsgen.q_calib(w, nq)
+    Qc = torch.from_numpy(qc.view(np.int16)).view(torch.bfloat16).cuda()
+    C = torch.empty((w.Hq, w.r), dtype=torch.int32, device="cuda")
+    imp = torch.empty((w.Hq, w.d), dtype=torch.float32, device="cuda")
+    dims = ds.Dims(w.B, w.Hq, w.Hkv, w.d, K.shape[2], w.r)
+    ws = ds.workspace(ds.OP_CALIBRATE, dims, w.T, nq, "cuda")
+    n0 = ds.kernel_launches()
+    ds.calibrate(Qc, K, C, w.T, importance=imp, ws=ws)
+    launches = ds.kernel_launches() - n0
+    ms = time_graph(lambda: ds.calibrate(Qc, K, C, w.T, importance=imp, ws=ws), steps, 5)
+    nbytes = w.B * w.Hkv * w.T * w.d * 2 + w.B * w.Hq * nq * w.d * 2
+    return {"us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm_peak,
+            "bytes": nbytes, "calibration_queries_per_head": nq, "launches": launches}
+
+
+def group_entry(w, inputs, hbm_peak, steps: int = 50):
+    """Group-shared selection on grouped KV heads: the step's label append,
+    ds_group_score_topk and ds_group_sparse_decode (one selection per KV group,
+    each kept row read once for the group's query heads)."""
+    import torch
+
+    import post_token_sparse_b200 as ds
+
+    Q, K, V = inputs
+    C = torch.from_numpy(dsgen.channels(w)).cuda()
+    label = torch.empty((w.B, w.Hq, w.T, w.r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(K, C, label, 0, w.T)
+    sg = torch.empty((w.B * w.Hkv, w.T), dtype=torch.float32, device="cuda")
+    idx = torch.empty((w.B * w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    ws = ds.workspace(ds.OP_GROUP_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
+
+    def step():
+        ds.label_append(K, C, label, w.T - 1, 1)
+        ds.group_score_topk(Q, C, label, sg, idx, w.T)
+        ds.group_sparse_decode(Q, K, V, idx, O, w.T, w.scale, ws=ws)
+
+    ms = time_graph(step, steps, 3)
+    nb = w.group_step_bytes()
+    return {"us_per_step": ms * 1e3, "bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": nb / (ms * 1e-3) / 1e9 / hbm_peak,
+            "tokens_heads_per_s": w.B * w.Hq * w.T / (ms * 1e-3)}
+
+
+def block_entry(w, inputs, hbm_peak, bs: int = 64, steps: int = 50):
+    """Block-granular selection with blocks of bs tokens and the same token budget
+    as the workload's k (kb = k / bs blocks): the step's label append,
+    ds_block_score_topk and ds_block_sparse_decode."""
+    import torch
+
+    import post_token_sparse_b200 as ds
+
+    Q, K, V = inputs
+    kb = max(1, w.k // bs)
+    C = torch.from_numpy(dsgen.channels(w)).cuda()
+    label = torch.empty((w.B, w.Hq, w.T, w.r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(K, C, label, 0, w.T)
+    BH = w.B * w.Hq
+    sb = torch.empty((BH, -(-w.T // bs)), dtype=torch.float32, device="cuda")
+    bidx = torch.empty((BH, kb), dtype=torch.int32, device="cuda")
+    O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    ws = ds.workspace(ds.OP_BLOCK_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, kb * bs, "cuda")
+
+    def step():
+        ds.label_append(K, C, label, w.T - 1, 1)
+        ds.block_score_topk(Q, C, label, sb, bidx, w.T, bs)
+        ds.block_sparse_decode(Q, K, V, bidx, O, w.T, bs, w.scale, ws=ws)
+
+    ms = time_graph(step, steps, 3)
+    nb = w.block_step_bytes(bs, kb)
+    return {"us_per_step": ms * 1e3, "block": bs, "blocks_kept": kb, "bytes": nb,
+            "gbs": nb / (ms * 1e-3) / 1e9, "frac_of_measured_hbm": nb / (ms * 1e-3) / 1e9 / hbm_peak,
+            "tokens_heads_per_s": w.B * w.Hq * w.T / (ms * 1e-3)}
 
 
 def _rounded(e):
@@ -502,6 +635,10 @@ def run_sweep(skip: str, hbm_peak: float):
         first_of_set = not name.startswith("sweep") or name.endswith("r8-k512")
         if first_of_set:
             e["dense"] = dense_entry(ww, max(10, n // 3), 2, hbm_peak, inputs=inp)
+        if ww.Hq > ww.Hkv:
+            e["group_shared"] = group_entry(ww, inp, hbm_peak)
+        if first_of_set and ww.T >= 16384:
+            e["block_select"] = block_entry(ww, inp, hbm_peak, steps=20)
         out[name] = _rounded(e)
         if name == dsgen.ORDER[-1] and name.startswith("sweep"):
             full = ww.with_(name="sweep-B32-H32-T32K-r128-kT", r=ww.d, k=ww.T)
@@ -603,6 +740,8 @@ def main():
         line["dense"] = dn
         line["speedup_vs_dense"] = dn["us_per_step"] / line["us_per_step"]
         line["cpu_baseline"] = time_oracle(base, args.cpu_seconds)
+        line["calibrate"] = _rounded(calib_entry(w, inputs[1], hbm_peak))
+        line["block_select"] = _rounded(block_entry(w, inputs, hbm_peak))
     del inputs
     torch.cuda.empty_cache()
     if rank == 0 and world == 1:

@@ -55,6 +55,19 @@ class Workload:
     def label_bytes(self) -> int:
         return self.B * self.Hq * self.T * self.r * 2
 
+    # Block-granular selection with kb blocks of bs tokens: every label row, the
+    # block scores written and read back, the kept blocks' K/V rows, Q and O.
+    def block_step_bytes(self, bs: int, kb: int) -> int:
+        nblk = -(-self.T // bs)
+        return (self.label_bytes() + self.B * self.Hq * (nblk * 4 * 2 + kb * 4
+                + kb * bs * 2 * self.d * 2 + self.d * 2 + self.d * 4))
+
+    # Group-shared selection: every label row, each kept K/V row once per KV
+    # group, the group scores written and read back, Q and O per query head.
+    def group_step_bytes(self) -> int:
+        return (self.label_bytes() + self.B * self.Hkv * self.k * (2 * self.d * 2 + 4)
+                + self.B * self.Hkv * self.T * 4 * 2 + self.B * self.Hq * (self.d * 2 + self.d * 4))
+
 
 _BASE_SEED = 0xD5000000
 

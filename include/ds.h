@@ -77,7 +77,10 @@ enum {
   DS_OP_SPARSE_DECODE = 3,
   DS_OP_DECODE = 4,
   DS_OP_SCORE_TOPK = 5,
-  DS_OP_DECODE_STEP = 6
+  DS_OP_DECODE_STEP = 6,
+  DS_OP_CALIBRATE = 7, /* k: calibration queries per head (Nq) */
+  DS_OP_GROUP_SPARSE_DECODE = 8,
+  DS_OP_BLOCK_SPARSE_DECODE = 9 /* k: kept rows = kb * bs */
 };
 
 /* Device status bits (ds_device_status). */
@@ -134,11 +137,14 @@ ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int3
                   void* ws, size_t ws_bytes, ds_stream_t stream);
 
 /*
- * ds_score_topk -- ds_score followed by ds_topk in one launch.
+ * ds_score_topk -- ds_score followed by ds_topk.
  *
- * Same results as the two calls (same fp32 scores, same index set), without
- * writing the scores to memory unless `scores` is non-NULL.  Limits as for
- * ds_topk.  Needs no workspace.
+ * Same results as the two calls (same fp32 scores, same index set).  With
+ * scores == NULL: one launch that computes the scores while selecting and
+ * never writes them.  With a scores buffer ([B*Hq, T] fp32, written): the same
+ * one launch, except for r >= 16 and T > 4096, where the scores are written
+ * first and the selection reads them (two launches; faster there).  Limits as
+ * for ds_topk.  Needs no workspace.
  */
 ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
                         int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream);
@@ -178,10 +184,12 @@ ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const in
  * Key design) and self-attention runs over those tokens only (Abstract).
  *
  * One CTA per query head performs the three phases on chip when r is 8, 16,
- * 32, 64 or 128, k <= 8192 and the head's selection fits one CTA; otherwise
- * the three calls are issued on `stream`.  idx: [B*Hq, k] int32 (required).
- * O and lse as for ds_sparse_decode; the attention's summation order may
- * differ from ds_sparse_decode's (fp32 rounding only).  ws:
+ * 32, 64 or 128, k <= 8192, B*Hq <= 296 (one wave of two CTAs per SM) and the
+ * head's selection fits one CTA; otherwise the three calls are issued on
+ * `stream` (the selection through a score buffer in the workspace when
+ * r >= 16 and T > 4096, see ds_score_topk).  idx: [B*Hq, k] int32
+ * (required).  O and lse as for ds_sparse_decode; the attention's summation
+ * order may differ from ds_sparse_decode's (fp32 rounding only).  ws:
  * ds_workspace_size(DS_OP_DECODE_STEP, dims, T, k) bytes, zero-filled before
  * first use (0 bytes when fused).  Other arguments as for the calls above.
  */
@@ -235,6 +243,101 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
 ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,
                                    const int32_t* idx, float* O, float* lse, ds_dims dims,
                                    int32_t T, int32_t k, float scale, ds_stream_t stream);
+
+/*
+ * ds_group_score_topk -- one token selection per KV group (grouped KV heads).
+ *
+ * The G = Hq/Hkv query heads of a group read the same K/V rows; selecting
+ * once per group lets each kept row be read once for all of them (token
+ * sparsity, Double Sparsity page, Abstract and Key points 2; the page gives
+ * no group score -- reading taken: the sum of the member heads' approximate
+ * scores).  group_scores[b*Hkv+g, t] = sum over h = g*G .. g*G+G-1, in that
+ * order, of the fp32 score ds_score gives for head h (same operation order),
+ * for t < T; idx[b*Hkv+g] = the k tokens of largest group score, ties to the
+ * lower index, ascending (as ds_topk).
+ *
+ * Q: [B,Hq,d] bf16.  C: [Hq,r] int32.  label: [B,Hq,T_cap,r] bf16.
+ * group_scores: [B*Hkv, T] fp32 (written; the caller's buffer).  idx:
+ * [B*Hkv, k] int32.  Requires r in {8,16,32,64,128}, G*r <= 12288,
+ * 1 <= k <= T <= min(T_cap, 1048576).  Two launches.
+ */
+ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
+                              float* group_scores, int32_t* idx, ds_dims dims, int32_t T,
+                              int32_t k, ds_stream_t stream);
+
+/*
+ * ds_group_sparse_decode -- attention over the group's kept tokens.
+ *
+ * As ds_sparse_decode, except that idx has one row per KV group
+ * ([B*Hkv, k], e.g. from ds_group_score_topk) and every query head of the
+ * group attends over its group's row.  The group's heads are adjacent in
+ * launch order, so a kept K/V row is fetched from HBM once and served to the
+ * other heads from L2.  ws: ds_workspace_size(DS_OP_GROUP_SPARSE_DECODE, dims,
+ * T, k) bytes, zero-filled before first use (left zero-filled).
+ */
+ds_status ds_group_sparse_decode(const void* Q, const void* K, const void* V,
+                                 const int32_t* idx, float* O, float* lse, ds_dims dims,
+                                 int32_t T, int32_t k, float scale, void* ws, size_t ws_bytes,
+                                 ds_stream_t stream);
+
+/*
+ * ds_block_score_topk -- block-granular token selection.
+ *
+ * Block informativeness (page "Jenga: Enhancing LLM Long-Context Fine-tuning
+ * with Contextual Token Sparsity", Core method 1: a token's informativeness
+ * counts positive scores only, a block's is the largest of its tokens';
+ * Observation 2: blocks of 64 tokens).  block_scores[bh, j] = max over the
+ * tokens t of block j (t in [j*bs, min((j+1)*bs, T))) of max(s[bh,t], 0), s
+ * the fp32 score of ds_score; bidx[bh] = the kb blocks of largest block score,
+ * ties to the lower block, ascending (a fixed count: the page keeps blocks
+ * against a threshold tuned per layer on a model).
+ *
+ * Q, C, label as for ds_score.  block_scores: [B*Hq, ceil(T/bs)] fp32
+ * (written).  bidx: [B*Hq, kb] int32.  Requires bs a power of two <= 64, r in
+ * {8,16,32,64,128}, 1 <= kb <= ceil(T/bs), T <= T_cap.  Two launches.
+ */
+ds_status ds_block_score_topk(const void* Q, const int32_t* C, const void* label,
+                              float* block_scores, int32_t* bidx, ds_dims dims, int32_t T,
+                              int32_t bs, int32_t kb, ds_stream_t stream);
+
+/*
+ * ds_block_sparse_decode -- attention over the tokens of the kept blocks.
+ *
+ * As ds_sparse_decode over the kb*bs rows of the blocks bidx[bh] ([B*Hq, kb],
+ * e.g. from ds_block_score_topk): row r is token bidx[bh, r/bs]*bs + r%bs;
+ * rows at or past T (the short last block) are skipped.  A block's rows are
+ * contiguous in K and V, so the gathers read whole runs of bs rows.  ws:
+ * ds_workspace_size(DS_OP_BLOCK_SPARSE_DECODE, dims, T, kb*bs) bytes,
+ * zero-filled before first use (left zero-filled).
+ */
+ds_status ds_block_sparse_decode(const void* Q, const void* K, const void* V,
+                                 const int32_t* bidx, float* O, float* lse, ds_dims dims,
+                                 int32_t T, int32_t bs, int32_t kb, float scale, void* ws,
+                                 size_t ws_bytes, ds_stream_t stream);
+
+/*
+ * ds_calibrate -- offline channel calibration: the label channels C.
+ *
+ * The channel pattern is static, so it is fixed offline from a calibration
+ * set (Double Sparsity page, Method details: Core idea and Technical
+ * framework); the page leaves the criterion open ("unknown", Key design).
+ * Reading taken: the importance of channel c for query head h is the mean,
+ * over every pair (calibration query n, cached token t < T) of the same
+ * sequence b, of |q[b,h,n,c] * k[b,g(h),t,c]|:
+ *   I[h,c] = sum_b (sum_n |q[b,h,n,c]|) * (sum_t |k[b,g(h),t,c]|) / (B*Nq*T),
+ * column sums in fp32 in a fixed order (deterministic).  C[h] holds the r
+ * channels of largest I[h,.] (ties to the lower channel), ascending -- the
+ * input ds_label_append expects.
+ *
+ * Qc: [B,Hq,Nq,d] bf16 calibration queries.  K: [B,Hkv,T_cap,d] bf16, rows
+ * t < T read.  C: [Hq, r] int32 out (r = dims.r).  importance: [Hq, d] fp32
+ * out, or NULL.  ws: ds_workspace_size(DS_OP_CALIBRATE, dims, T, Nq) bytes of
+ * device memory (scratch; no contents required).  Requires 1 <= T <= T_cap,
+ * Nq >= 1, 1 <= r <= d.  Two launches, no host synchronisation.
+ */
+ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_dims dims, int32_t T,
+                       int32_t* C, float* importance, void* ws, size_t ws_bytes,
+                       ds_stream_t stream);
 
 /*
  * Bytes of device workspace `op` needs for these sizes (0 if none).  Depends

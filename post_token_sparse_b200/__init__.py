@@ -33,7 +33,7 @@ LIB_PATH = os.path.join(_HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
 (OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK,
- OP_DECODE_STEP) = range(7)
+ OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE) = range(10)
 DEV_BAD_CHANNEL, DEV_BAD_INDEX = 1, 2
 
 
@@ -73,6 +73,13 @@ def _load():
         "ds_device_status": [u32p, i32, vp],
         "ds_decode_step": [vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, i32,
                            vp, ctypes.c_size_t, vp],
+        "ds_calibrate": [vp, i32, vp, Dims, i32, vp, vp, vp, ctypes.c_size_t, vp],
+        "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
+        "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
+        "ds_block_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, i32, ctypes.c_float,
+                                   vp, ctypes.c_size_t, vp],
+        "ds_group_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, vp,
+                                   ctypes.c_size_t, vp],
     }
     for name, args in sig.items():
         if not hasattr(lib, name):
@@ -228,6 +235,73 @@ def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):
                           _ptr(V, torch.bfloat16, "V"), _ptr(O, torch.float32, "O"),
                           _ptr(lse, torch.float32, "lse"), dims, T, scale,
                           _ptr(ws, None, "ws"), nbytes, _stream(Q.device)), "ds_decode")
+
+
+def group_score_topk(Q, C, label, group_scores, idx, T: int):
+    """One selection per KV group: group_scores [B*Hkv, T] fp32, idx [B*Hkv, k]."""
+    B, Hq, T_cap, r = label.shape
+    Hkv = group_scores.shape[0] // B
+    dims = Dims(B, Hq, Hkv, Q.shape[-1], T_cap, r)
+    _check(_lib.ds_group_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
+                                    _ptr(label, torch.bfloat16, "label"),
+                                    _ptr(group_scores, torch.float32, "group_scores"),
+                                    _ptr(idx, torch.int32, "idx"), dims, T, idx.shape[-1],
+                                    _stream(Q.device)), "ds_group_score_topk")
+
+
+def group_sparse_decode(Q, K, V, idx, O, T: int, scale: float, lse=None, ws=None):
+    """Attention of every query head over its KV group's kept tokens (idx [B*Hkv, k])."""
+    dims = dims_of(Q, K, 1)
+    k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_GROUP_SPARSE_DECODE, dims, T, k, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_group_sparse_decode(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+                                       _ptr(V, torch.bfloat16, "V"), _ptr(idx, torch.int32, "idx"),
+                                       _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"),
+                                       dims, T, k, scale, _ptr(ws, None, "ws"), nbytes,
+                                       _stream(Q.device)), "ds_group_sparse_decode")
+
+
+def block_score_topk(Q, C, label, block_scores, bidx, T: int, bs: int):
+    """Block-granular selection: block_scores [B*Hq, ceil(T/bs)] fp32, bidx [B*Hq, kb]."""
+    B, Hq, T_cap, r = label.shape
+    dims = Dims(B, Hq, Hq, Q.shape[-1], T_cap, r)
+    _check(_lib.ds_block_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
+                                    _ptr(label, torch.bfloat16, "label"),
+                                    _ptr(block_scores, torch.float32, "block_scores"),
+                                    _ptr(bidx, torch.int32, "bidx"), dims, T, bs, bidx.shape[-1],
+                                    _stream(Q.device)), "ds_block_score_topk")
+
+
+def block_sparse_decode(Q, K, V, bidx, O, T: int, bs: int, scale: float, lse=None, ws=None):
+    """Attention of every query head over the tokens of its kept blocks."""
+    dims = dims_of(Q, K, 1)
+    kb = bidx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_BLOCK_SPARSE_DECODE, dims, T, kb * bs, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_block_sparse_decode(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+                                       _ptr(V, torch.bfloat16, "V"), _ptr(bidx, torch.int32, "bidx"),
+                                       _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"),
+                                       dims, T, bs, kb, scale, _ptr(ws, None, "ws"), nbytes,
+                                       _stream(Q.device)), "ds_block_sparse_decode")
+
+
+def calibrate(Qc, K, C, T: int, importance=None, ws=None):
+    """Offline channel calibration: C [Hq, r] from calibration queries Qc
+    [B,Hq,Nq,d] and keys K [B,Hkv,T_cap,d] (tokens < T); importance [Hq, d]
+    fp32 optionally."""
+    B, Hq, Nq, d = Qc.shape
+    _, Hkv, T_cap, _ = K.shape
+    dims = Dims(B, Hq, Hkv, d, T_cap, C.shape[1])
+    if ws is None:
+        ws = workspace(OP_CALIBRATE, dims, T, Nq, Qc.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_calibrate(_ptr(Qc, torch.bfloat16, "Qc"), Nq, _ptr(K, torch.bfloat16, "K"),
+                             dims, T, _ptr(C, torch.int32, "C"),
+                             _ptr(importance, torch.float32, "importance"),
+                             _ptr(ws, None, "ws"), nbytes, _stream(Qc.device)), "ds_calibrate")
 
 
 def device_status(clear: bool = True, device=None) -> int:

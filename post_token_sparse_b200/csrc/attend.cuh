@@ -42,11 +42,18 @@ struct AttnParams {
   float* lse;      // optional
   float* partial;      // [BH, S, kPartialStride] when S > 1
   uint32_t* arrivals;  // [BH] split-arrival counters (zero between calls) when S > 1
+  int idx_per_group;   // idx rows per KV head ([B*Hkv, rows]) instead of per query head
+  int block;           // > 0: idx holds block ids ([.., rows/block]); row r is token
+                       // idx[r/block]*block + r%block, rows at or past T skipped
   int Hq, Hkv, T_cap, T;
   int rows;           // k (sparse) or T (dense)
   int rows_per_split; // multiple of 4
   float scale_log2;   // softmax scale * log2(e)
 };
+
+__device__ __forceinline__ int nb_total(const AttnParams& p) {
+  return (p.T + p.block - 1) / p.block;
+}
 
 __device__ __forceinline__ float dot8(const uint4& v, const float* q) {
   float a = bf_lo(v.x) * q[0];
@@ -97,14 +104,29 @@ k_attend(const AttnParams p) {
   const int g = lane >> 3, c = lane & 7;
 
   if constexpr (kSparse) {
-    const int32_t* src = p.idx + (size_t)bh * p.rows + r0;
-    for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
-      int t = src[i];
-      if (t < 0 || t >= p.T) {
-        flag_status(2u);
-        t = min(max(t, 0), p.T - 1);
+    if (p.block) {
+      const int nb = p.rows / p.block;
+      const int32_t* src = p.idx + (size_t)bh * nb;
+      for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
+        const int r = r0 + i;
+        int b = src[r / p.block];
+        if (b < 0 || b >= nb_total(p)) {
+          flag_status(2u);
+          b = min(max(b, 0), nb_total(p) - 1);
+        }
+        const int t = b * p.block + r % p.block;
+        idx_s[i] = t < p.T ? t : -1;  // the short last block
       }
-      idx_s[i] = t;
+    } else {
+      const int32_t* src = p.idx + (size_t)(p.idx_per_group ? bkv : bh) * p.rows + r0;
+      for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
+        int t = src[i];
+        if (t < 0 || t >= p.T) {
+          flag_status(2u);
+          t = min(max(t, 0), p.T - 1);
+        }
+        idx_s[i] = t;
+      }
     }
     __syncthreads();
   }
@@ -136,7 +158,8 @@ k_attend(const AttnParams p) {
   auto issue = [&](int step) {
     const int lr = w_begin + step * 4 + g;  // row within the split
     if (lr < w_end) {
-      const int t = kSparse ? idx_s[lr] : r0 + lr;
+      int t = kSparse ? idx_s[lr] : r0 + lr;
+      if (kSparse && t < 0) t = 0;  // a skipped row: any valid address
       const uint4* krow = reinterpret_cast<const uint4*>(Kh + (size_t)t * kHeadDim);
       const uint4* vrow = reinterpret_cast<const uint4*>(Vh + (size_t)t * kHeadDim);
       uint4* st = my_ring + (step % kAttnStages) * kAttnStageU4 + g * 32;
@@ -169,7 +192,8 @@ k_attend(const AttnParams p) {
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 4);
-    if (w_begin + n * 4 + g < w_end) {
+    const int lr = w_begin + n * 4 + g;
+    if (lr < w_end && (!kSparse || idx_s[lr] >= 0)) {
       float a = 1.f;
       if (x > m) {
         a = exp2f(m - x);  // 0 when m is still -inf

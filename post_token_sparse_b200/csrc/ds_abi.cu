@@ -14,6 +14,7 @@
 #include "ds.h"
 
 #include "attend.cuh"
+#include "calib.cuh"
 #include "common.cuh"
 #include "label.cuh"
 #include "score.cuh"
@@ -246,7 +247,8 @@ ds_status check_attend_ws(const ds_dims& d, int rows, bool sparse, const void* w
 
 ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const void* V,
                         const int32_t* idx, float* O, float* lse, int T, int rows, float scale,
-                        void* ws, cudaStream_t st) {
+                        void* ws, cudaStream_t st, bool idx_per_group = false,
+                        int block = 0) {
   const bool sparse = idx != nullptr;
   const int BH = d.B * d.Hq;
   const SplitPlan sp = plan_splits(BH, rows, sparse);
@@ -256,6 +258,8 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
   p.K = static_cast<const uint16_t*>(K);
   p.V = static_cast<const uint16_t*>(V);
   p.idx = idx;
+  p.idx_per_group = idx_per_group ? 1 : 0;
+  p.block = block;
   p.O = O;
   p.lse = lse;
   p.partial = static_cast<float*>(ws);
@@ -282,10 +286,24 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
 // The fused step applies when r has a vector path, the head's selection fits
 // one CTA, k is small enough for its index list to stay in shared memory, and
 // the whole layout fits a CTA's shared memory.  Depends only on the sizes.
+// Selection from the label cache: one fused launch (scores computed while
+// selecting), or, for r >= 16 on heads longer than one sample, the scores
+// written first and the selection run over them.  The second needs a score
+// buffer but measured faster there: the score kernel streams the labels once
+// at full rate, and the selection's passes then read 4 bytes a token.
+bool prefer_score_then_select(int r, int T) { return r >= 16 && T > kSample; }
+
+// The one-launch step runs every head's whole chain in one CTA at two CTAs per
+// SM.  That pays while all heads fit one wave; with more heads the separate
+// kernels (three top-k CTAs and six attention CTAs per SM) hide each other's
+// latency better, so the step falls back to them.
+constexpr int kStepMaxHeads = 2 * 148;
+
 bool step_fused(const ds_dims& d, int T, int k, int* chunk_out, size_t* smem_out) {
   const int r = d.r;
   if (!(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) return false;
   if (k > kStepMaxK) return false;
+  if (d.B * d.Hq > kStepMaxHeads) return false;
   TopkPlan tp;
   if (!plan_topk(d.B * d.Hq, T, k, &tp) || tp.cs != 1) return false;
   const size_t smem = StepLayout(tp.chunk, k).bytes();
@@ -293,6 +311,21 @@ bool step_fused(const ds_dims& d, int T, int k, int* chunk_out, size_t* smem_out
   *chunk_out = tp.chunk;
   *smem_out = smem;
   return true;
+}
+
+// Workspace of the separate-kernels step: the attention's split partials and
+// counters, then (when the selection runs over written scores) [BH, T] fp32
+// scores.  Returns the total; *scores_off gets the offset of the scores (0: none).
+size_t step_fallback_ws(const ds_dims& d, int T, int k, size_t* scores_off) {
+  const int BH = d.B * d.Hq;
+  size_t n = partial_bytes(BH, plan_splits(BH, k, true));
+  size_t off = 0;
+  if (prefer_score_then_select(d.r, T)) {
+    off = (n + 255) & ~(size_t)255;
+    n = off + (((size_t)BH * T * sizeof(float) + 255) & ~(size_t)255);
+  }
+  if (scores_off) *scores_off = off;
+  return n;
 }
 
 template <int R>
@@ -334,7 +367,19 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
       int chunk;
       size_t smem;
       if (step_fused(dims, T, k, &chunk, &smem)) return 0;
+      return step_fallback_ws(dims, T, k, nullptr);
+    }
+    case DS_OP_BLOCK_SPARSE_DECODE:  // k: kept rows, blocks x block size
+      if (k < 1) return 0;
       return partial_bytes(BH, plan_splits(BH, k, true));
+    case DS_OP_GROUP_SPARSE_DECODE:  // the same split plan as the per-head call
+      if (k < 1 || k > T) return 0;
+      return partial_bytes(BH, plan_splits(BH, k, true));
+    case DS_OP_CALIBRATE: {
+      if (k < 1) return 0;  // k: calibration queries per head
+      const size_t nck = (T + kAbsumRows - 1) / kAbsumRows, ncq = (k + kAbsumRows - 1) / kAbsumRows;
+      const size_t bytes = ((size_t)dims.B * dims.Hkv * nck + (size_t)BH * ncq) * kHeadDim * 4;
+      return (bytes + 255) & ~(size_t)255;
     }
     default:
       return 0;
@@ -413,6 +458,11 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
   if (s != DS_OK) return s;
   auto Qb = static_cast<const uint16_t*>(Q);
   auto Lb = static_cast<const uint16_t*>(label);
+  if (scores && prefer_score_then_select(dims.r, T)) {
+    s = launch_score(Qb, C, Lb, scores, dims, T, stream);
+    if (s != DS_OK) return s;
+    return launch_topk(ScoresSource{scores}, idx, dims.B * dims.Hq, T, k, stream);
+  }
   switch (dims.r) {
     case 8: return fused_topk<8>(Qb, C, Lb, scores, idx, dims, T, k, stream);
     case 16: return fused_topk<16>(Qb, C, Lb, scores, idx, dims, T, k, stream);
@@ -535,9 +585,11 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
   int chunk = 0;
   size_t smem = 0;
   const bool fused = step_fused(dims, T, k, &chunk, &smem);
+  size_t scores_off = 0;
   if (!fused) {
     s = check_attend_ws(dims, k, true, ws, ws_bytes);
     if (s != DS_OK) return s;
+    if (ws_bytes < step_fallback_ws(dims, T, k, &scores_off)) return DS_ERR_WORKSPACE;
     const bool vec = dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 ||
                      dims.r == 128;
     if (!vec) return DS_ERR_UNSUPPORTED;  // the fused score+select needs a vector path
@@ -575,7 +627,163 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
     s = ds_label_append(K, C, label, dims, T - 1, 1, stream);
     if (s != DS_OK) return s;
   }
-  s = ds_score_topk(Q, C, label, nullptr, idx, dims, T, k, stream);
+  float* scores = scores_off ? reinterpret_cast<float*>(static_cast<char*>(ws) + scores_off)
+                             : nullptr;
+  s = ds_score_topk(Q, C, label, scores, idx, dims, T, k, stream);
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
+}
+
+extern "C" ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_dims dims,
+                                  int32_t T, int32_t* C, float* importance, void* ws,
+                                  size_t ws_bytes, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Qc || !K || !C || !aligned16(Qc) || !aligned16(K) || !aligned16(C))
+    return DS_ERR_INVALID_ARG;
+  if (importance && !aligned16(importance)) return DS_ERR_INVALID_ARG;
+  if (Nq < 1 || T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
+  const int nck = (T + kAbsumRows - 1) / kAbsumRows, ncq = (Nq + kAbsumRows - 1) / kAbsumRows;
+  if (nck > 65535 || ncq > 65535) return DS_ERR_UNSUPPORTED;
+  const size_t need = ds_workspace_size(DS_OP_CALIBRATE, dims, T, Nq);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return DS_ERR_WORKSPACE;
+  float* pk = static_cast<float*>(ws);
+  float* pq = pk + (size_t)dims.B * dims.Hkv * nck * kHeadDim;
+  if ((int64_t)dims.B * (dims.Hkv + dims.Hq) > 65535) return DS_ERR_UNSUPPORTED;
+  k_absum<<<dim3(std::max(nck, ncq), dims.B * (dims.Hkv + dims.Hq)), kAbsumThreads, 0, stream>>>(
+      static_cast<const uint16_t*>(K), (size_t)dims.T_cap * kHeadDim, T, dims.B * dims.Hkv, pk,
+      static_cast<const uint16_t*>(Qc), (size_t)Nq * kHeadDim, Nq, pq);
+  s = launched();
+  if (s != DS_OK) return s;
+  const float inv_pairs = (float)(1.0 / ((double)dims.B * (double)Nq * (double)T));
+  k_calib_select<<<dims.Hq, kHeadDim, 0, stream>>>(pk, nck, pq, ncq, dims.B, dims.Hq, dims.Hkv,
+                                                   dims.r, inv_pairs, C, importance);
+  return launched();
+}
+
+namespace {
+
+template <int R>
+ds_status launch_group_score(const uint16_t* Q, const int32_t* C, const uint16_t* label,
+                             float* sg, const ds_dims& d, int T, cudaStream_t st) {
+  using S = ScoreShape<R>;
+  const int G = d.Hq / d.Hkv;
+  dim3 grid((T + S::kTokensPerCta - 1) / S::kTokensPerCta, d.B * d.Hkv);
+  k_group_score<R><<<grid, kScoreThreads, (size_t)G * R * sizeof(float), st>>>(
+      Q, C, label, sg, d.Hq, d.Hkv, d.T_cap, T);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
+                                         float* group_scores, int32_t* idx, ds_dims dims,
+                                         int32_t T, int32_t k, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !C || !label || !group_scores || !idx || !aligned16(Q) || !aligned16(C) ||
+      !aligned16(label) || !aligned16(group_scores) || !aligned16(idx))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
+  const int G = dims.Hq / dims.Hkv;
+  if ((size_t)G * dims.r * sizeof(float) > 48 * 1024) return DS_ERR_UNSUPPORTED;
+  if (!(dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 || dims.r == 128))
+    return DS_ERR_UNSUPPORTED;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  auto Qb = static_cast<const uint16_t*>(Q);
+  auto Lb = static_cast<const uint16_t*>(label);
+  switch (dims.r) {
+    case 8: s = launch_group_score<8>(Qb, C, Lb, group_scores, dims, T, stream); break;
+    case 16: s = launch_group_score<16>(Qb, C, Lb, group_scores, dims, T, stream); break;
+    case 32: s = launch_group_score<32>(Qb, C, Lb, group_scores, dims, T, stream); break;
+    case 64: s = launch_group_score<64>(Qb, C, Lb, group_scores, dims, T, stream); break;
+    case 128: s = launch_group_score<128>(Qb, C, Lb, group_scores, dims, T, stream); break;
+    default: return DS_ERR_UNSUPPORTED;
+  }
+  if (s != DS_OK) return s;
+  return launch_topk(ScoresSource{group_scores}, idx, dims.B * dims.Hkv, T, k, stream);
+}
+
+extern "C" ds_status ds_group_sparse_decode(const void* Q, const void* K, const void* V,
+                                            const int32_t* idx, float* O, float* lse,
+                                            ds_dims dims, int32_t T, int32_t k, float scale,
+                                            void* ws, size_t ws_bytes, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  s = check_attend_ws(dims, k, true, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream, true);
+}
+
+namespace {
+
+bool block_size_ok(int bs) { return bs >= 1 && bs <= 64 && (bs & (bs - 1)) == 0; }
+
+template <int R>
+ds_status launch_block_score(const uint16_t* Q, const int32_t* C, const uint16_t* label,
+                             float* sb, const ds_dims& d, int T, int bs, cudaStream_t st) {
+  using S = ScoreShape<R>;
+  dim3 grid((T + S::kTokensPerCta - 1) / S::kTokensPerCta, d.B * d.Hq);
+  k_block_score<R><<<grid, kScoreThreads, 0, st>>>(Q, C, label, sb, d.Hq, d.T_cap, T, bs);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" ds_status ds_block_score_topk(const void* Q, const int32_t* C, const void* label,
+                                         float* block_scores, int32_t* bidx, ds_dims dims,
+                                         int32_t T, int32_t bs, int32_t kb, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !C || !label || !block_scores || !bidx || !aligned16(Q) || !aligned16(C) ||
+      !aligned16(label) || !aligned16(block_scores) || !aligned16(bidx))
+    return DS_ERR_INVALID_ARG;
+  if (!block_size_ok(bs)) return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
+  const int nblk = (T + bs - 1) / bs;
+  if (kb < 1 || kb > nblk) return DS_ERR_INVALID_ARG;
+  if (!(dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 || dims.r == 128))
+    return DS_ERR_UNSUPPORTED;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  auto Qb = static_cast<const uint16_t*>(Q);
+  auto Lb = static_cast<const uint16_t*>(label);
+  switch (dims.r) {
+    case 8: s = launch_block_score<8>(Qb, C, Lb, block_scores, dims, T, bs, stream); break;
+    case 16: s = launch_block_score<16>(Qb, C, Lb, block_scores, dims, T, bs, stream); break;
+    case 32: s = launch_block_score<32>(Qb, C, Lb, block_scores, dims, T, bs, stream); break;
+    case 64: s = launch_block_score<64>(Qb, C, Lb, block_scores, dims, T, bs, stream); break;
+    default: s = launch_block_score<128>(Qb, C, Lb, block_scores, dims, T, bs, stream); break;
+  }
+  if (s != DS_OK) return s;
+  return launch_topk(ScoresSource{block_scores}, bidx, dims.B * dims.Hq, nblk, kb, stream);
+}
+
+extern "C" ds_status ds_block_sparse_decode(const void* Q, const void* K, const void* V,
+                                            const int32_t* bidx, float* O, float* lse,
+                                            ds_dims dims, int32_t T, int32_t bs, int32_t kb,
+                                            float scale, void* ws, size_t ws_bytes,
+                                            ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !bidx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(bidx) || !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (!block_size_ok(bs)) return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
+  if (kb < 1 || kb > (T + bs - 1) / bs) return DS_ERR_INVALID_ARG;
+  const int rows = kb * bs;
+  s = check_attend_ws(dims, rows, true, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  return launch_attend(dims, Q, K, V, bidx, O, lse, T, rows, scale, ws, stream, false, bs);
 }

@@ -129,3 +129,116 @@ k_score_any(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
 }
 
 }  // namespace ds
+
+namespace ds {
+
+// Group scores for grouped KV heads: sg[b,g,t] = sum over the G query heads
+// h = g*G .. g*G+G-1 of s[b,h,t], each s computed exactly as k_score_vec
+// computes it and the sum taken in head order in fp32 (group-shared
+// selection: one top-k per KV group, so that each selected K/V row is read
+// once for all of the group's query heads).
+// grid: (ceil(T / kTokensPerCta), B*Hkv); dynamic shared memory G*R floats.
+template <int R>
+__global__ void __launch_bounds__(kScoreThreads)
+k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
+              const uint16_t* __restrict__ label, float* __restrict__ sg, int Hq, int Hkv,
+              int T_cap, int T) {
+  using S = ScoreShape<R>;
+  extern __shared__ __align__(16) float qg[];  // [G][R]
+  const int G = Hq / Hkv;
+  const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+  for (int i = threadIdx.x; i < G * R; i += blockDim.x) {
+    const int hh = i / R, j = i % R;
+    const int h = g * G + hh;
+    int c = C[h * R + j];
+    if (c < 0 || c >= kHeadDim) {
+      flag_status(1u);
+      c &= (kHeadDim - 1);
+    }
+    qg[i] = bf_at(Q + (size_t)(b * Hq + h) * kHeadDim + c);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = lane % S::kLanes;
+  auto token = [&](int i) {
+    return blockIdx.x * S::kTokensPerCta + (warp * S::kSlots + i) * S::kRowsPerInstr +
+           lane / S::kLanes;
+  };
+  float acc[S::kSlots];
+  for (int hh = 0; hh < G; ++hh) {
+    const uint4* lab =
+        reinterpret_cast<const uint4*>(label + (size_t)(b * Hq + g * G + hh) * T_cap * R);
+    uint4 v[S::kSlots];
+#pragma unroll
+    for (int i = 0; i < S::kSlots; ++i) {
+      const int t = token(i);
+      v[i] = t < T ? ldg_stream(lab + (size_t)t * S::kLanes + chunk) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < S::kSlots; ++i) {
+      const float s = lane_group_score<R>(v[i], qg + hh * R, chunk);  // all lanes take part
+      acc[i] = hh == 0 ? s : acc[i] + s;
+    }
+  }
+  float* out = sg + (size_t)bg * T;
+#pragma unroll
+  for (int i = 0; i < S::kSlots; ++i) {
+    const int t = token(i);
+    if (t < T && chunk == 0) out[t] = acc[i];
+  }
+}
+
+}  // namespace ds
+
+namespace ds {
+
+// Block informativeness for block-granular selection (page "Jenga: Enhancing
+// LLM Long-Context Fine-tuning with Contextual Token Sparsity", Core method 1:
+// a token's informativeness counts positive scores only; a block's is the
+// largest of its tokens').  sb[bh, j] = max over t in block j (bs tokens,
+// clipped to T) of max(s[bh, t], 0), s computed exactly as k_score_vec does.
+// grid: (ceil(T / kTokensPerCta), BH); bs a power of two <= 64 (it divides the
+// tile); scores staged in shared memory, then one warp reduces 32 tokens (or
+// one 64-token block) per pass.
+template <int R>
+__global__ void __launch_bounds__(kScoreThreads)
+k_block_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
+              const uint16_t* __restrict__ label, float* __restrict__ sb, int Hq, int T_cap, int T,
+              int bs) {
+  using S = ScoreShape<R>;
+  __shared__ __align__(16) float qs[R];
+  __shared__ float sc[S::kTokensPerCta];
+  const int bh = blockIdx.y, h = bh % Hq;
+  load_qc(Q, C, bh, h, R, qs);
+  __syncthreads();
+  const uint4* lab = reinterpret_cast<const uint4*>(label + (size_t)bh * T_cap * R);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = lane % S::kLanes;
+  const int t0 = blockIdx.x * S::kTokensPerCta;
+  auto row = [&](int i) { return (warp * S::kSlots + i) * S::kRowsPerInstr + lane / S::kLanes; };
+  uint4 v[S::kSlots];
+#pragma unroll
+  for (int i = 0; i < S::kSlots; ++i) {
+    const int t = t0 + row(i);
+    v[i] = t < T ? ldg_stream(lab + (size_t)t * S::kLanes + chunk) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < S::kSlots; ++i) {
+    const float s = lane_group_score<R>(v[i], qs, chunk);  // all lanes take part
+    if (chunk == 0) sc[row(i)] = t0 + row(i) < T ? fmaxf(s, 0.f) : 0.f;
+  }
+  __syncthreads();
+  const int nblk = (T + bs - 1) / bs;
+  float* out = sb + (size_t)bh * nblk;
+  const int step = bs > 32 ? bs : 32;  // tokens per warp pass
+  for (int base = warp * step; base < S::kTokensPerCta; base += kScoreThreads / 32 * step) {
+    float x = sc[base + lane];
+    if (bs > 32) x = fmaxf(x, sc[base + 32 + lane]);
+    const int seg = bs > 32 ? 32 : bs;  // lanes reduced together
+    for (int o = 1; o < seg; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    const int j = (t0 + base + lane) / bs;
+    if ((lane & (seg - 1)) == 0 && (bs > 32 ? lane == 0 : true) && j < nblk) out[j] = x;
+  }
+}
+
+}  // namespace ds

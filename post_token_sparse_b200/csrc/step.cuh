@@ -191,8 +191,10 @@ k_step(const StepParams p, int chunk) {
   uint16_t* over16 = reinterpret_cast<uint16_t*>(sm + SL.over);
   int32_t* idx_s = reinterpret_cast<int32_t*>(sm + SL.idx);
 
-  // 1. the newest token's label row
-  if (p.append) {
+  // 1. the newest token's label row, and q at the label channels (one load of
+  //    each channel id serves both)
+  float* qs = reinterpret_cast<float*>(sm + TopkLayout(chunk, 1).small + 64);
+  {
     const int t = p.T - 1;
     const uint16_t* krow = p.K + ((size_t)bkv * p.T_cap + t) * kHeadDim;
     uint16_t* lrow = p.label + ((size_t)bh * p.T_cap + t) * R;
@@ -202,21 +204,23 @@ k_step(const StepParams p, int chunk) {
         flag_status(1u);
         ch &= (kHeadDim - 1);
       }
-      const uint16_t v = krow[ch];
-      over16[j] = v;
-      lrow[j] = v;
+      qs[j] = bf_at(p.Q + (size_t)bh * kHeadDim + ch);
+      if (p.append) {
+        const uint16_t v = krow[ch];
+        over16[j] = v;
+        lrow[j] = v;
+      }
     }
-    __syncthreads();
   }
 
-  // 2. selection
+  // 2. selection (its first barrier publishes qs and the new row)
   LabelSource<R> src{p.Q, p.C, p.label, nullptr, p.Hq, p.T_cap};
   if (p.append) {
     src.over_t = p.T - 1;
     src.over_row = reinterpret_cast<const uint4*>(over16);
   }
   topk_body(src, sm, 1, 0, bh, p.T, p.k, chunk, p.idx ? p.idx + (size_t)bh * p.k : nullptr,
-            idx_s);
+            idx_s, true);
   __syncthreads();
 
   // 3. attention over the kept rows (the selection's shared memory is free now)

@@ -13,10 +13,11 @@
 //               blocks of 32 consecutive tokens spread over [0, T), or every
 //               token when T <= 4096.  Every CTA of a cluster draws the same
 //               sample, so all of them agree on what follows without talking.
-//   2. bracket  radix select on the sample: with the whole head sampled, the
-//               exact k-th key (lo = hi = threshold); otherwise the sample's
-//               keys at ranks k*m/T -/+ (5 standard deviations + 2) become
-//               hi / lo: keys above hi are selected, keys below lo are not.
+//   2. bracket  list select on the sample (below): with the whole head sampled,
+//               the exact k-th key (lo = hi = threshold), and the head's keys
+//               are classified on the way; otherwise the sample's keys at
+//               ranks k*m/T -/+ (5 standard deviations + 2) become hi / lo:
+//               keys above hi are selected, keys below lo are not.
 //   3. stream   one pass over this CTA's keys (computed from the label cache,
 //               or read from the scores): key > hi sets a bit of the "above"
 //               mask; lo <= key <= hi sets a bit of the "equal" mask when
@@ -26,10 +27,16 @@
 //               refinement takes over: one histogram pass per key digit
 //               narrows the bracket to the bin holding the k-th key and the
 //               stream pass repeats; a one-value bracket always fits.
-//   5. resolve  radix select of the remaining rank over the candidate lists
-//               (histograms merged over the cluster) gives the exact threshold
-//               key; candidates above it join the "above" mask, candidates
-//               equal to it the "equal" mask.
+//   5. resolve  select of the remaining rank over the candidates (a list
+//               select for one CTA; a radix select with histograms merged over
+//               the cluster otherwise) gives the exact threshold key;
+//               candidates above it join the "above" mask, candidates equal to
+//               it the "equal" mask.
+//
+// List select: radix select over 11-bit digits in which, after each digit, the
+// items of the chosen bin are compacted into a short list, so that the next
+// digit and the end touch only those; once at most one item per thread is
+// left, threads count the items above and equal to each.
 //   6. write    per-warp counts, a cluster-wide exclusive scan (pushed into the
 //               later CTAs before a barrier), then one 32-token group per lane:
 //               indices in ascending order, ties taken in index order.
@@ -55,6 +62,11 @@ constexpr int kSample = 4096;                // sample size (the whole head when
 constexpr int kSampleBlocks = kSample / 32;  // 128 blocks of 32 consecutive tokens
 constexpr int kCandCap = 4096;               // candidate list of one CTA
 constexpr float kBracketSigmas = 5.f;
+constexpr int kListCap = 1024;            // items of one list-select buffer
+constexpr int kRankCount = kTopkThreads;  // items at which ranks are counted directly
+constexpr int kSelectIters = 4;           // list select sources: 4 x (4 items per thread)
+constexpr int kWideBits = 13;             // sample histogram of one CTA: top 13 key bits
+constexpr int kWideBins = 1 << kWideBits;
 
 // digits of the 32-bit key: bits 31..21, 20..10, 9..0
 __host__ __device__ constexpr int digit_shift(int d) { return d == 0 ? 21 : (d == 1 ? 10 : 0); }
@@ -64,7 +76,7 @@ constexpr int kBinsPerThread = 2048 / kTopkThreads;  // 8
 
 // Shared-memory layout in 32-bit words (depends on the chunk and cluster size).
 struct TopkLayout {
-  int merged0, merged1, small, masks, X, words;
+  int merged0, merged1, small, masks, X, lists, words;
   __host__ __device__ TopkLayout(int chunk, int cs) {
     int o = 2048;  // histogram (2048 bins) at 0
     merged0 = o;   // cluster-merged histograms (CTA-local copies)
@@ -79,17 +91,35 @@ struct TopkLayout {
     X = o;  // candidates: keys [kCandCap], tokens [kCandCap]; while sampling, the
             // sample keys in the first half and two histograms in the second
     o += 2 * kCandCap;
+    // list select: two buffers of kListCap (key, token) pairs; with a cluster
+    // they overlay the merged histograms, which are not in use while a CTA
+    // selects on its own
+    if (cs > 1) {
+      lists = merged0;
+    } else {
+      lists = o;
+      o += 4 * kListCap;
+    }
     words = o;
   }
   __host__ __device__ size_t bytes() const { return (size_t)words * 4; }
 };
 static_assert(kSample <= kCandCap, "sample keys live in the candidate-key half");
-static_assert(2 * 2048 <= kCandCap, "two sample histograms live in the token half");
+static_assert(4 * kListCap == 2 * 2048, "list buffers fit the two merged histograms");
+static_assert(kCandCap + 4 * kListCap == kWideBins,
+              "the wide sample histogram spans the candidate tokens and the lists");
+static_assert(kRankCount == kTopkThreads, "one counted item per thread");
+static_assert(kBinsPerThread == 8, "find_bins reads its bins as two 16-byte vectors");
+static_assert(4 * kSelectIters * kTopkThreads >= kCandCap &&
+                  4 * kSelectIters * kTopkThreads >= kSample,
+              "every list select source fits the unrolled pass");
 
 enum {
   M_BIN = 0, M_ABOVE = 1, M_CNT = 2,     // find_bins, target 1
   M_BIN2 = 3, M_ABOVE2 = 4, M_CNT2 = 5,  // find_bins, target 2
   M_NCAND = 6,                           // this CTA's candidate count
+  M_LIST = 7,                            // list select: compaction counter (zero between uses)
+  M_THR = 14, M_NEED = 15,               // list select: result key, its rank among equal keys
   M_TOT = 8,                             // cluster totals: above, equal, cand, overflow
   M_GT_BEFORE = 12, M_EQ_BEFORE = 13     // counts of the earlier CTAs of the cluster
 };
@@ -101,7 +131,9 @@ __device__ __forceinline__ void cluster_or_cta_sync(int cs) {
     __syncthreads();
 }
 
-// Exclusive block-wide prefix sum over threads in thread order.
+// Exclusive block-wide prefix sum over threads in thread order.  One barrier;
+// scratch[0..kTopkWarps) must not be written again before the caller's next
+// barrier.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
@@ -114,38 +146,112 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   __syncthreads();
   uint32_t wbase = 0;
   for (int w = 0; w < warp; ++w) wbase += scratch[w];
-  __syncthreads();
   return wbase + incl - v;
 }
 
 // For rank r (1 = largest) finds the bin b (bins counted from the top) with
 // count(bins > b) < r <= count(bins >= b) and writes b, count(bins > b) and
-// count(b) to out[0..2]; r == 0 finds nothing.
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t r,
-                                         uint32_t* scratch, uint32_t* out) {
+// count(b) to out[0..2]; r == 0 finds nothing.  Two ranks share one scan.
+__device__ __forceinline__ void find_bins(const uint32_t* hist, int nbins, uint32_t r1,
+                                          uint32_t r2, uint32_t* scratch, uint32_t* out1,
+                                          uint32_t* out2) {
   uint32_t c[kBinsPerThread];
   uint32_t sum = 0;
+  const int top = nbins - 1 - threadIdx.x * kBinsPerThread;  // this thread's first bin
+  if ((nbins & 7) == 0) {
+    // bins top-7 .. top, 16-byte aligned: two vector loads
+    if (top >= 7) {
+      const uint4 lo = *reinterpret_cast<const uint4*>(hist + top - 7);
+      const uint4 hi = *reinterpret_cast<const uint4*>(hist + top - 3);
+      c[0] = hi.w; c[1] = hi.z; c[2] = hi.y; c[3] = hi.x;
+      c[4] = lo.w; c[5] = lo.z; c[6] = lo.y; c[7] = lo.x;
+    } else {
 #pragma unroll
-  for (int j = 0; j < kBinsPerThread; ++j) {
-    const int b = nbins - 1 - (threadIdx.x * kBinsPerThread + j);
-    c[j] = b >= 0 ? hist[b] : 0u;
-    sum += c[j];
-  }
-  const uint32_t above = block_exclusive_scan(sum, scratch);
-  if (r && sum > 0 && above < r && r <= above + sum) {
-    uint32_t acc = above;
+      for (int j = 0; j < kBinsPerThread; ++j) c[j] = 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kBinsPerThread; ++j) sum += c[j];
+  } else {
 #pragma unroll
     for (int j = 0; j < kBinsPerThread; ++j) {
-      if (acc + c[j] >= r) {
-        out[0] = (uint32_t)(nbins - 1 - (threadIdx.x * kBinsPerThread + j));
-        out[1] = acc;
-        out[2] = c[j];
-        break;
-      }
-      acc += c[j];
+      const int b = top - j;
+      c[j] = b >= 0 ? hist[b] : 0u;
+      sum += c[j];
     }
   }
+  const uint32_t above = block_exclusive_scan(sum, scratch);
+  auto find = [&](uint32_t r, uint32_t* out) {
+    if (r && sum > 0 && above < r && r <= above + sum) {
+      uint32_t acc = above;
+#pragma unroll
+      for (int j = 0; j < kBinsPerThread; ++j) {
+        if (acc + c[j] >= r) {
+          out[0] = (uint32_t)(nbins - 1 - (threadIdx.x * kBinsPerThread + j));
+          out[1] = acc;
+          out[2] = c[j];
+          break;
+        }
+        acc += c[j];
+      }
+    }
+  };
+  find(r1, out1);
+  find(r2, out2);
   __syncthreads();
+}
+
+// find_bins over NB * kTopkThreads bins, NB per thread (read as vectors).
+template <int NB>
+__device__ __forceinline__ void find_bins_wide(const uint32_t* hist, uint32_t r1, uint32_t r2,
+                                               uint32_t* scratch, uint32_t* out1,
+                                               uint32_t* out2) {
+  static_assert(NB % 16 == 0, "bins are read sixteen at a time");
+  const int topb = NB * kTopkThreads - 1 - NB * (int)threadIdx.x;  // this thread's highest bin
+  const uint4* v = reinterpret_cast<const uint4*>(hist + topb - (NB - 1));
+  uint32_t sum = 0;
+  // neighbouring threads' ranges are NB words apart: a rotated vector order
+  // keeps the eight lanes of each shared-memory wavefront on distinct banks
+#pragma unroll
+  for (int q = 0; q < NB / 4; ++q) {
+    const uint4 x = v[(q + threadIdx.x) % (NB / 4)];
+    sum += x.x + x.y + x.z + x.w;
+  }
+  const uint32_t above = block_exclusive_scan(sum, scratch);
+  auto find = [&](uint32_t r, uint32_t* out) {
+    if (r && sum > 0 && above < r && r <= above + sum) {
+      // this thread's bins, four vectors at a time from the top
+      uint32_t acc = above;
+      bool done = false;
+#pragma unroll
+      for (int q0 = NB / 4 - 4; q0 >= 0 && !done; q0 -= 4) {
+        uint4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = v[q0 + u];
+#pragma unroll
+        for (int u = 3; u >= 0; --u) {
+          const uint32_t c4[4] = {x[u].w, x[u].z, x[u].y, x[u].x};  // descending bins
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (!done && acc + c4[e] >= r) {
+              out[0] = (uint32_t)(topb - (NB - 1) + 4 * (q0 + u) + 3 - e);
+              out[1] = acc;
+              out[2] = c4[e];
+              done = true;
+            }
+            if (!done) acc += c4[e];
+          }
+        }
+      }
+    }
+  };
+  find(r1, out1);
+  find(r2, out2);
+  __syncthreads();
+}
+
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t r,
+                                         uint32_t* scratch, uint32_t* out) {
+  find_bins(hist, nbins, r, 0u, scratch, out, out);
 }
 
 // hist (nbins bins) summed over the cluster into every CTA's merged copy;
@@ -274,56 +380,202 @@ struct LabelSource {
   }
 };
 
-// Keys of rank r1 and r2 (1 = largest; 0 = not wanted) among keys[0..m), by a
-// three-digit radix select.  hist already holds the digit-0 histogram; hist2
-// has room for two 2048-bin histograms.
-__device__ __forceinline__ void sample_ranks(const uint32_t* keys, int m, const uint32_t* hist,
-                                             uint32_t* hist2, uint32_t* misc, uint32_t r1,
-                                             uint32_t r2, uint32_t& key1, uint32_t& key2) {
-  uint32_t* scratch = misc + 48;
-  uint32_t p1 = 0, p2 = 0;
-  for (int d = 0; d < 3; ++d) {
-    const int nb = digit_bins(d);
-    const uint32_t* h1 = hist;
-    const uint32_t* h2 = hist;
-    if (d > 0) {
-      for (int i = threadIdx.x; i < 2 * nb; i += kTopkThreads) hist2[i] = 0u;
+// List select: the key of rank r (1 = largest) among the live items of a key
+// array in shared memory.  Source item i < n has key key0[i] and token tok0(i);
+// the live items are those that carry the prefix pf above bit `top` (top = 32:
+// every item), and r is at most their number.  When the caller already has the
+// first digit's bin, the count above it and its count (first_bin >= 0; the
+// digit is first_bits wide), the first histogram is skipped.  With kCls, live items above the result set
+// their token's bit in gtm and live items equal to it in eqm (tokens of
+// [c0, c0 + len) only; bit t - c0); kSeqTok: tok0(i) == i, and c0 is a multiple
+// of 32.  n <= 4 * kSelectIters * kTopkThreads, key0 16-byte aligned, and key0
+// readable up to n rounded up to 4.  need: the result's rank among the
+// keys equal to it.  misc[M_LIST] is zero on entry and on exit.  Block-uniform.
+template <bool kCls, bool kSeqTok, class TokFn>
+__device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0, int n, int top,
+                                                uint32_t pf, uint32_t r, int first_bits,
+                                                int first_bin, uint32_t first_above,
+                                                uint32_t first_cnt,
+                                                uint32_t* hist, uint32_t* lists, uint32_t* misc,
+                                                uint32_t* gtm, uint32_t* eqm, int c0, int len,
+                                                uint32_t& need) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t* sk = key0;
+  const uint32_t* st = nullptr;  // tokens of the current list (null: the source array)
+  int ns = n, buf = 0;
+  auto token = [&](int i) -> int { return st ? (int)st[i] : tok0(i); };
+  auto mark = [&](uint32_t* m, int t) {
+    const int j = t - c0;
+    if (j >= 0 && j < len) atomicOr(&m[j >> 5], 1u << (j & 31));
+  };
+  auto live = [&](uint32_t key) { return top >= 32 || (key >> top) == pf; };
+
+  while (!(st && ns <= kRankCount) && top > 0) {
+    const int bits = first_bin >= 0 ? first_bits : (top < 11 ? top : 11);
+    const int sh = top - bits;
+    const uint32_t nb = 1u << bits;
+    uint32_t bin, above, cnt;
+    if (first_bin >= 0) {
+      bin = (uint32_t)first_bin;
+      above = first_above;
+      cnt = first_cnt;
+      first_bin = -1;
+    } else {
+      for (int i = threadIdx.x; i < (int)nb; i += kTopkThreads) hist[i] = 0u;
       __syncthreads();
-      const int hs = digit_shift(d - 1), sh = digit_shift(d);
-      for (int i = threadIdx.x; i < m; i += kTopkThreads) {
-        const uint32_t key = keys[i];
-        if (r1 && (key >> hs) == p1) atomicAdd(&hist2[(key >> sh) & (nb - 1)], 1u);
-        if (r2 && (key >> hs) == p2) atomicAdd(&hist2[nb + ((key >> sh) & (nb - 1))], 1u);
+      for (int i = threadIdx.x; i < ns; i += kTopkThreads) {
+        const uint32_t key = sk[i];
+        if (live(key)) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
       }
       __syncthreads();
-      h1 = hist2;
-      h2 = hist2 + nb;
+      find_bin(hist, (int)nb, r, misc + 48, misc + M_BIN);
+      bin = misc[M_BIN];
+      above = misc[M_ABOVE];
+      cnt = misc[M_CNT];
     }
-    find_bin(h1, nb, r1, scratch, misc + M_BIN);
-    find_bin(h2, nb, r2, scratch, misc + M_BIN2);
-    if (r1) {
-      p1 = (p1 << digit_bits(d)) | misc[M_BIN];
-      r1 -= misc[M_ABOVE];
+    r -= above;
+    const bool compact = cnt <= (uint32_t)kListCap;
+    uint32_t* dk = lists + buf * 2 * kListCap;
+    uint32_t* dt = dk + kListCap;
+    // One pass, four consecutive items per thread and load: items above the
+    // bin are marked, the bin's items flagged (4 bits per load, in registers);
+    // then one slot reservation per warp and the flagged items are copied.
+    uint32_t keep = 0u;  // bit 4*it + u: item it*4*kTopkThreads + 4*threadIdx.x + u
+#pragma unroll
+    for (int it = 0; it < kSelectIters; ++it) {
+      if (it * 4 * kTopkThreads < ns) {
+        const int i0 = it * 4 * kTopkThreads + 4 * threadIdx.x;
+        const uint4 kv = *reinterpret_cast<const uint4*>(sk + i0);
+        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t up = 0u;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool lv = i0 + u < ns && live(kk[u]);
+          const uint32_t dg = (kk[u] >> sh) & (nb - 1);
+          if (lv && dg > bin) up |= 1u << u;
+          if (lv && dg == bin) keep |= 1u << (4 * it + u);
+        }
+        if (kCls) {
+          if (kSeqTok && !st) {
+            // tokens i0..i0+3; eight lanes make one 32-token mask word
+            uint32_t wm = up << (4 * (lane & 7));
+            wm |= __shfl_xor_sync(0xffffffffu, wm, 1);
+            wm |= __shfl_xor_sync(0xffffffffu, wm, 2);
+            wm |= __shfl_xor_sync(0xffffffffu, wm, 4);
+            const int j = i0 - 4 * (lane & 7) - c0;
+            if ((lane & 7) == 0 && wm && j >= 0 && j < len) gtm[j >> 5] |= wm;
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if ((up >> u) & 1u) mark(gtm, token(i0 + u));
+          }
+        }
+      }
     }
-    if (r2) {
-      p2 = (p2 << digit_bits(d)) | misc[M_BIN2];
-      r2 -= misc[M_ABOVE2];
+    if (compact) {
+      const uint32_t c = __popc(keep);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      uint32_t base = 0u;
+      if (lane == 31 && incl) base = atomicAdd(&misc[M_LIST], incl);
+      base = __shfl_sync(0xffffffffu, base, 31) + incl - c;
+      while (keep) {
+        const int b = __ffs(keep) - 1;
+        keep &= keep - 1u;
+        const int i = (b >> 2) * 4 * kTopkThreads + 4 * threadIdx.x + (b & 3);
+        dk[base] = sk[i];
+        if (kCls) dt[base] = (uint32_t)token(i);
+        ++base;
+      }
+      // zero keys (below every key of a non-NaN score) pad the list to a
+      // multiple of 64 for the rank count
+      if (threadIdx.x < 64 && cnt + threadIdx.x < (uint32_t)kListCap) dk[cnt + threadIdx.x] = 0u;
     }
     __syncthreads();
+    pf = (pf << bits) | bin;
+    top = sh;
+    if (compact) {
+      sk = dk;
+      st = dt;
+      ns = (int)cnt;
+      buf ^= 1;
+      if (threadIdx.x == 0) misc[M_LIST] = 0u;  // next used after a barrier
+    }
   }
-  key1 = p1;
-  key2 = p2;
+
+  uint32_t thr;
+  if (st && ns <= kRankCount) {
+    // Each item's count of larger and of equal keys, split over P threads
+    // when the list is short; the list is zero-padded to a multiple of 64.
+    const int P = ns <= 64 ? 4 : (ns <= 128 ? 2 : 1);
+    const int per = kTopkThreads / P;
+    const int i = threadIdx.x % per, part = threadIdx.x / per;
+    const int span = ((ns + 63) & ~63) / P;
+    uint32_t* pgt = lists + buf * 2 * kListCap;  // the list buffer not in use
+    uint32_t* peq = pgt + kTopkThreads;
+    if (i < ns) {
+      const uint32_t mine = sk[i];
+      uint32_t gt = 0u, eq = 0u;
+      const uint4* v = reinterpret_cast<const uint4*>(sk + part * span);
+      for (int j = 0; j < span / 4; j += 4) {
+        const uint4 x[4] = {v[j], v[j + 1], v[j + 2], v[j + 3]};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gt += (x[q].x > mine ? 1u : 0u) + (x[q].y > mine ? 1u : 0u) +
+                (x[q].z > mine ? 1u : 0u) + (x[q].w > mine ? 1u : 0u);
+          eq += (x[q].x == mine ? 1u : 0u) + (x[q].y == mine ? 1u : 0u) +
+                (x[q].z == mine ? 1u : 0u) + (x[q].w == mine ? 1u : 0u);
+        }
+      }
+      pgt[threadIdx.x] = gt;
+      peq[threadIdx.x] = eq;
+    }
+    __syncthreads();
+    if (threadIdx.x < ns) {
+      uint32_t gt = 0u, eq = 0u;
+      for (int q = 0; q < P; ++q) {
+        gt += pgt[q * per + threadIdx.x];
+        eq += peq[q * per + threadIdx.x];
+      }
+      if (gt < r && r <= gt + eq) {  // every thread holding the result's value
+        misc[M_THR] = sk[threadIdx.x];
+        misc[M_NEED] = r - gt;
+      }
+    }
+    __syncthreads();
+    thr = misc[M_THR];
+    need = misc[M_NEED];
+  } else {  // every bit fixed: the live items all equal the prefix
+    thr = pf;
+    need = r;
+  }
+  if (kCls) {
+    for (int i = threadIdx.x; i < ns; i += kTopkThreads) {
+      const uint32_t key = sk[i];
+      if (!live(key)) continue;
+      if (key > thr)
+        mark(gtm, token(i));
+      else if (key == thr)
+        mark(eqm, token(i));
+    }
+  }
+  __syncthreads();
+  return thr;
 }
 
 // The streaming passes of the kernel below.
 
-// Sample pass: keys of the m sampled tokens into keys[], their digit-0
-// histogram into hist; scores of this CTA's tokens when the whole head is the
-// sample.
+// Sample pass: keys of the m sampled tokens into keys[], the histogram of
+// their top 32 - hshift bits into hist; scores of this CTA's tokens when the
+// whole head is the sample.
 template <class Source>
 __device__ __forceinline__ void sample_pass(const Source& src, int bh, int T, int m, bool whole,
-                                         uint32_t* keys, uint32_t* hist, float* scores_out,
-                                         int c0, int len, const float* qs) {
+                                         uint32_t* keys, uint32_t* hist, int hshift,
+                                         float* scores_out, int c0, int len, const float* qs) {
   const int q32 = T >> 5;
   auto tok = [whole, q32](int j) {
     return whole ? j : ((int)((long long)(j >> 5) * q32 / kSampleBlocks) << 5) + (j & 31);
@@ -332,7 +584,7 @@ __device__ __forceinline__ void sample_pass(const Source& src, int bh, int T, in
              [&](bool v, int j, uint32_t key, float s) {
                if (v) {
                  keys[j] = key;
-                 atomicAdd(&hist[key >> digit_shift(0)], 1u);
+                 atomicAdd(&hist[key >> hshift], 1u);
                  if (whole && scores_out && j >= c0 && j < c0 + len) scores_out[j] = s;
                }
              },
@@ -390,11 +642,12 @@ __device__ __forceinline__ void digit_hist_pass(const Source& src, int bh, int T
 // The selection of one head by one CTA of its cluster (cs CTAs, this one of
 // rank `rank`, shared memory `sm` laid out by TopkLayout(chunk, cs)).  The
 // selected indices, ascending, go to dst_g (global, k entries) and/or dst_s
-// (shared memory, k entries); either may be null.
+// (shared memory, k entries); either may be null.  qs_ready: the caller has
+// already written the source's query values (TopkLayout::small + 64 onwards).
 template <class Source>
 __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int cs, int rank,
                                           int bh, int T, int k, int chunk, int32_t* dst_g,
-                                          int32_t* dst_s) {
+                                          int32_t* dst_s, bool qs_ready = false) {
   const TopkLayout L(chunk, cs);
   uint32_t* hist = sm;
   uint32_t* misc = sm + L.small;
@@ -404,7 +657,7 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
   uint32_t* gtm = sm + L.masks;
   uint32_t* eqm = gtm + chunk / 32;
   uint32_t* cand_key = sm + L.X;  // also the sample keys while sampling
-  uint32_t* cand_tok = cand_key + kCandCap;  // also two histograms while sampling
+  uint32_t* cand_tok = cand_key + kCandCap;
 
   const int c0 = min(rank * chunk, T);
   const int len = min(chunk, T - c0);
@@ -414,33 +667,64 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
 
   for (int i = threadIdx.x; i < L.small + 64; i += kTopkThreads) sm[i] = 0u;
   for (int i = threadIdx.x; i < 2 * (chunk / 32); i += kTopkThreads) gtm[i] = 0u;
-  src.prepare(bh, qs);
+  if (cs == 1) {  // the wide sample histogram (below)
+    uint4* z = reinterpret_cast<uint4*>(cand_tok);
+    for (int i = threadIdx.x; i < kWideBins / 4; i += kTopkThreads) z[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (!qs_ready) src.prepare(bh, qs);
   // every CTA of the cluster is running and its counters are zero before any
   // remote access
   cluster_or_cta_sync(cs);
 
   // ---- 1. sample ---------------------------------------------------------------
+  // one CTA: a 13-bit histogram over the candidate-token half and the lists
+  // (free until the bracket is known); a cluster: the 11-bit one
   const bool whole = T <= kSample;
   const int m = whole ? T : kSample;
-  sample_pass(src, bh, T, m, whole, cand_key, hist, scores_out, c0, len, qs);
+  const bool wide = cs == 1;
+  uint32_t* hist0 = wide ? cand_tok : hist;
+  const int hbits = wide ? kWideBits : digit_bits(0);
+  sample_pass(src, bh, T, m, whole, cand_key, hist0, 32 - hbits, scores_out, c0, len, qs);
   __syncthreads();
 
   // ---- 2. bracket ----------------------------------------------------------------
   uint32_t lo, hi;
+  uint32_t* lists = sm + L.lists;
+  uint32_t need_unused;
   if (whole) {
-    uint32_t thr, unused;
-    sample_ranks(cand_key, m, hist, cand_tok, misc, (uint32_t)k, 0u, thr, unused);
+    // exact threshold over every key of the head; this CTA's tokens are
+    // classified on the way
+    if (wide)
+      find_bins_wide<kWideBins / kTopkThreads>(hist0, (uint32_t)k, 0u, misc + 48, misc + M_BIN,
+                                               misc + M_BIN);
+    else
+      find_bin(hist0, 2048, (uint32_t)k, misc + 48, misc + M_BIN);
+    const int b0 = (int)misc[M_BIN];
+    const uint32_t a0 = misc[M_ABOVE], n0 = misc[M_CNT];
+    const uint32_t thr = list_select<true, true>(
+        cand_key, [](int i) { return i; }, T, 32, 0u, (uint32_t)k, hbits, b0, a0, n0, hist,
+        lists, misc, gtm, eqm, c0, len, need_unused);
     lo = hi = thr;
   } else {
     const float e = (float)k * (float)m / (float)T;
     const float sd = sqrtf(e * (1.f - (float)k / (float)T));
     const float margin = kBracketSigmas * sd + 2.f;
     const int r_hi = (int)floorf(e - margin), r_lo = (int)ceilf(e + margin);
-    uint32_t khi, klo;
-    sample_ranks(cand_key, m, hist, cand_tok, misc, r_hi >= 1 ? (uint32_t)r_hi : 0u,
-                 r_lo <= m ? (uint32_t)r_lo : 0u, khi, klo);
-    hi = r_hi >= 1 ? khi : 0xffffffffu;
-    lo = r_lo <= m ? klo : 0u;
+    const uint32_t rh = r_hi >= 1 ? (uint32_t)r_hi : 0u, rl = r_lo <= m ? (uint32_t)r_lo : 0u;
+    if (wide)
+      find_bins_wide<kWideBins / kTopkThreads>(hist0, rh, rl, misc + 48, misc + M_BIN,
+                                               misc + M_BIN2);
+    else
+      find_bins(hist0, 2048, rh, rl, misc + 48, misc + M_BIN, misc + M_BIN2);
+    const int bh0 = (int)misc[M_BIN], bl0 = (int)misc[M_BIN2];
+    const uint32_t ah = misc[M_ABOVE], nh = misc[M_CNT], al = misc[M_ABOVE2], nl = misc[M_CNT2];
+    auto no_tok = [](int) { return 0; };
+    hi = rh ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rh, hbits, bh0, ah, nh, hist,
+                                        lists, misc, gtm, eqm, c0, len, need_unused)
+            : 0xffffffffu;
+    lo = rl ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rl, hbits, bl0, al, nl, hist,
+                                        lists, misc, gtm, eqm, c0, len, need_unused)
+            : 0u;
   }
 
   // ---- 3/4. stream and check; exact refinement if the bracket fails -----------
@@ -448,14 +732,8 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
   uint32_t prefix = 0, krem = (uint32_t)k;
   for (;;) {
     const bool one = lo == hi;
-    if (whole) {
-      // every key of the head is in cand_key (the sample): this CTA's range;
-      // the bracket is exact here, so no candidate is listed over them
-      for (int j = threadIdx.x; j < len; j += kTopkThreads) {
-        const uint32_t key = cand_key[c0 + j];
-        if (key > hi) atomicOr(&gtm[j >> 5], 1u << (j & 31));
-        else if (key == hi) atomicOr(&eqm[j >> 5], 1u << (j & 31));
-      }
+    if (whole && level == 0) {
+      // classified by the select above
     } else {
       classify_pass(src, bh, T, c0, len, lo, hi, level == 0 ? scores_out : nullptr, gtm, eqm,
                     cand_key, cand_tok, &misc[M_NCAND], qs);
@@ -521,7 +799,15 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
 
   // ---- 5. resolve within the bracket -------------------------------------------
   uint32_t need = krem;
-  if (lo != hi) {
+  if (lo != hi && cs == 1) {
+    // the candidates share the bits of lo and hi above their highest differing bit
+    const uint32_t ncand = misc[M_NCAND];
+    const int top = 32 - __clz(lo ^ hi);
+    list_select<true, false>(
+        cand_key, [&](int i) { return c0 + (int)cand_tok[i]; }, (int)ncand, top,
+        top >= 32 ? 0u : lo >> top, krem, 0, -1, 0u, 0u, hist, lists, misc, gtm, eqm, c0, len,
+        need);
+  } else if (lo != hi) {
     const uint32_t ncand = misc[M_NCAND];
     uint32_t p = 0, r = krem;
     for (int d = 0; d < 3; ++d) {

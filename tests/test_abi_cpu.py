@@ -153,6 +153,86 @@ def test_workspace_sizes():
         lib.ds_workspace_size(ds.OP_DECODE, d, 262144, 1)
 
 
+def test_decode_step_fuses_only_one_wave_of_heads():
+    lib = ds.lib()
+    # one launch (no workspace) while B*Hq <= 2 x 148; the separate kernels beyond
+    assert lib.ds_workspace_size(ds.OP_DECODE_STEP, _dims(B=8, Hq=32, Hkv=32, T_cap=4096), 4096,
+                                 256) == 0
+    assert lib.ds_workspace_size(ds.OP_DECODE_STEP, _dims(B=9, Hq=32, Hkv=32, T_cap=4096), 4096,
+                                 256) == 0
+    assert lib.ds_workspace_size(ds.OP_DECODE_STEP, _dims(B=10, Hq=32, Hkv=32, T_cap=4096),
+                                 4096, 256) > 0
+    assert lib.ds_workspace_size(ds.OP_DECODE_STEP, _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8),
+                                 32768, 2048) > 0
+
+
+def test_group_calls_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
+    mis = ctypes.c_void_p(FAKE + 4)
+    assert lib.ds_group_score_topk(P, P, P, NUL, P, d, 100, 10, NUL) == bad  # scores required
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 100, 101, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 1001, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, mis, P, d, 100, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(Hq=6, Hkv=4), 100, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(r=12), 100, 10, NUL) == \
+        ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_group_sparse_decode(P, P, P, P, P, NUL, d, 100, 101, 1.0, NUL, 0, NUL) == bad
+    assert lib.ds_group_sparse_decode(P, P, P, NUL, P, NUL, d, 100, 10, 1.0, NUL, 0, NUL) == bad
+    # the same split plan (and workspace) as the per-head attention
+    dl = _dims(B=1, Hq=32, Hkv=8, T_cap=262144, r=8)
+    assert lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384) == \
+        lib.ds_workspace_size(ds.OP_SPARSE_DECODE, dl, 262144, 16384) > 0
+    need = lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384)
+    assert lib.ds_group_sparse_decode(P, P, P, P, P, NUL, dl, 262144, 16384, 1.0, P, need - 1,
+                                      NUL) == ds.DS_ERR_WORKSPACE
+
+
+def test_block_calls_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
+    for bs in (0, 3, 128, -64):
+        assert lib.ds_block_score_topk(P, P, P, P, P, d, 1000, bs, 1, NUL) == bad
+        assert lib.ds_block_sparse_decode(P, P, P, P, P, NUL, d, 1000, bs, 1, 1.0, NUL, 0,
+                                          NUL) == bad
+    assert lib.ds_block_score_topk(P, P, P, P, P, d, 1000, 64, 17, NUL) == bad  # 16 blocks
+    assert lib.ds_block_score_topk(P, P, P, P, P, d, 1000, 64, 0, NUL) == bad
+    assert lib.ds_block_score_topk(P, P, P, NUL, P, d, 1000, 64, 4, NUL) == bad
+    assert lib.ds_block_score_topk(P, P, P, P, P, d, 1001, 64, 4, NUL) == bad
+    assert lib.ds_block_score_topk(P, P, P, P, P, _dims(r=12), 1000, 64, 4, NUL) == \
+        ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_block_sparse_decode(P, P, P, P, P, NUL, d, 1000, 64, 17, 1.0, NUL, 0, NUL) == bad
+    dl = _dims(B=1, Hq=4, Hkv=4, T_cap=262144, r=8)
+    need = lib.ds_workspace_size(ds.OP_BLOCK_SPARSE_DECODE, dl, 262144, 256 * 64)
+    assert need == lib.ds_workspace_size(ds.OP_SPARSE_DECODE, dl, 262144, 256 * 64) > 0
+    assert lib.ds_block_sparse_decode(P, P, P, P, P, NUL, dl, 262144, 64, 256, 1.0, P, need - 1,
+                                      NUL) == ds.DS_ERR_WORKSPACE
+
+
+def test_calibrate_validation_and_workspace():
+    lib = ds.lib()
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=5000, r=16)
+    bad = ds.DS_ERR_INVALID_ARG
+    mis = ctypes.c_void_p(FAKE + 4)
+    need = lib.ds_workspace_size(ds.OP_CALIBRATE, d, 5000, 16)
+    # key chunk sums [B*Hkv][ceil(T/512)][128] + query sums [B*Hq][1][128], fp32, 256-rounded
+    assert need == ((2 * 2 * 10 + 2 * 8 * 1) * 128 * 4 + 255) // 256 * 256
+    assert lib.ds_workspace_size(ds.OP_CALIBRATE, d, 5000, 0) == 0
+    assert lib.ds_calibrate(P, 16, P, d, 5000, P, NUL, P, need - 1, NUL) == ds.DS_ERR_WORKSPACE
+    assert lib.ds_calibrate(P, 16, P, d, 5000, P, NUL, NUL, 0, NUL) == ds.DS_ERR_WORKSPACE
+    assert lib.ds_calibrate(P, 0, P, d, 5000, P, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, d, 0, P, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, d, 5001, P, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(NUL, 16, P, d, 5000, P, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, d, 5000, mis, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, d, 5000, P, mis, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, _dims(r=129), 500, P, NUL, P, need, NUL) == bad
+    assert lib.ds_calibrate(P, 16, P, _dims(d=64, r=8), 500, P, NUL, P, need, NUL) == \
+        ds.DS_ERR_UNSUPPORTED
+
+
 def test_launch_counter_starts_untouched():
     assert ds.kernel_launches() >= 0
 
