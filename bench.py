@@ -8,7 +8,7 @@ batch: append the new token's label row, score every cached token on the
 label channels and keep the top k, then exact attention over the kept rows --
 one ds_decode_step call (one launch where the sizes allow; the same step as
 separate calls is timed beside it for per-kernel stage times).  Inputs are seeded and synthetic (``dsgen``) and resident
-in HBM; the step is one CUDA graph; L2 is flushed (256 MiB written) between
+in HBM; the step is one CUDA graph; L2 is flushed (256 MiB written, then read) between
 steps and each step is timed with CUDA events, so every step reads its bytes
 from HBM.
 
@@ -42,6 +42,16 @@ METRIC = "sparse decode µs/step & HBM GB/s (% of 8 TB/s) vs dense, T=1K–256K"
 FLUSH_BYTES = 256 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic_llama2-7b-B8-H32-T4K.txt")
 CSRC = os.path.join(ROOT, "post_token_sparse_b200", "csrc")
+
+
+def flush_l2(buf):
+    """Evict L2 between timed steps: write a buffer larger than L2, then read it
+    back, so that L2 holds clean lines (a write alone leaves about 126 MB of dirty
+    lines whose write-back would be charged to the next timed kernel)."""
+    import torch
+
+    buf.zero_()
+    torch.sum(buf.view(torch.int64), dtype=torch.int64)
 
 
 def parse():
@@ -268,7 +278,7 @@ class Step:
 
     def timed(self):
         """One step after an L2 flush: (step ms, [stage ms])."""
-        self.flush.zero_()
+        flush_l2(self.flush)
         self.graph.replay()
         self.torch.cuda.synchronize()
         ev = self.events
@@ -355,11 +365,11 @@ def time_e2e(step: Step, steps: int, warmup: int):
         return e0.elapsed_time(e1)
 
     for _ in range(warmup):
-        step.flush.zero_()
+        flush_l2(step.flush)
         one()
     tot = 0.0
     for _ in range(steps):
-        step.flush.zero_()
+        flush_l2(step.flush)
         tot += one()
     h2d = q_h.numel() * 2 + 2 * kv_h[0].numel() * 2
     return tot, h2d, o_h.numel() * 4
@@ -496,7 +506,7 @@ def dense_entry(w, steps, warmup, hbm_peak, inputs=None):
 
 def time_graph(fn, steps: int, warmup: int) -> float:
     """Mean device ms of fn() (a few launches) replayed as a CUDA graph, with the
-    L2 flushed (256 MiB write) before each replay."""
+    L2 flushed (256 MiB written, then read back) before each replay."""
     import torch
 
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -510,11 +520,11 @@ def time_graph(fn, steps: int, warmup: int) -> float:
         fn()
         e1.record()
     for _ in range(warmup):
-        flush.zero_()
+        flush_l2(flush)
         g.replay()
     tot = 0.0
     for _ in range(steps):
-        flush.zero_()
+        flush_l2(flush)
         g.replay()
         torch.cuda.synchronize()
         tot += e0.elapsed_time(e1)
@@ -714,7 +724,8 @@ def main():
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
                        "T": w.T, "r": w.r, "k": w.k, "path": args.mode,
                        "fused_score_topk": not args.unfused,
-                       "l2": "flushed between steps (256 MiB write)", "cuda_graph": True,
+                       "l2": "flushed between steps (256 MiB written, then read back)",
+                       "cuda_graph": True,
                        "parallelism": f"replicas x{world}"},
             "stages": stages, "roofline": roofline,
             "gpu_launches": step.launches_per_step * args.steps,

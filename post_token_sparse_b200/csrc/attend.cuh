@@ -96,12 +96,21 @@ k_attend(const AttnParams p) {
   const int b = bkv / p.Hkv;
   const int h = (bkv % p.Hkv) * G + blockIdx.x;
   const int bh = b * p.Hq + h;
-  const int S = gridDim.y, split = blockIdx.y;
+  // Split s of KV head bkv runs in grid slot (s - 5*bkv) mod S: CTAs resident
+  // together then work on different key ranges of their heads, instead of every
+  // head's same range (head strides in K and V are large powers of two).
+  const int S = gridDim.y;
+  const int split = (int)((blockIdx.y + 5u * (unsigned)bkv) % (unsigned)S);
   const int r0 = split * p.rows_per_split;
   const int nrows = min(p.rows_per_split, p.rows - r0);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 3, c = lane & 7;
+
+  // this lane's query chunks, issued before the index staging so that the two
+  // loads overlap
+  const uint4* qrow = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim);
+  const uint4 qa = qrow[c], qb = qrow[8 + c];
 
   if constexpr (kSparse) {
     if (p.block) {
@@ -134,9 +143,7 @@ k_attend(const AttnParams p) {
   // this lane's 16 query values, pre-scaled into the log2 domain
   float q[16];
   {
-    const uint4* qrow = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim);
-    const uint4 a = qrow[c], bq = qrow[8 + c];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+    const uint32_t w[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       q[2 * i] = bf_lo(w[i]) * p.scale_log2;

@@ -159,8 +159,9 @@ struct TopkPlan {
 // head anyway).  Longer heads are cut so that one CTA's expected number of
 // candidates -- the tokens inside the sample bracket -- stays near half its
 // list, and, with few heads, further (down to kTopkMinKeys tokens per CTA) to
-// give every SM four CTAs.
+// fill one wave of the cluster grid.
 constexpr int kTopkMinKeys = 2048;
+constexpr int kTopkClusterWave = 384;
 
 bool plan_topk(int BH, int T, int k, TopkPlan* out) {
   int cs = (T + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
@@ -170,8 +171,11 @@ bool plan_topk(int BH, int T, int k, TopkPlan* out) {
     const double frac = 2.0 * (kBracketSigmas * std::sqrt(e * (1.0 - p)) + 3.0) / kSample;
     const double max_chunk = 0.5 * kCandCap / std::max(frac, 1e-9);
     cs = std::max(cs, (int)std::min<double>(kMaxCluster, std::ceil(T / max_chunk)));
-    if (BH * cs < 4 * 148) {
-      const int want = (4 * 148 + BH - 1) / BH;
+    // few heads: spread each over more CTAs, up to one wave.  Clusters are
+    // placed whole inside a GPC, so at three selection CTAs per SM about 384
+    // CTAs of clusters run at once; a second wave would double the time.
+    if (BH * cs < kTopkClusterWave) {
+      const int want = std::max(1, kTopkClusterWave / BH);
       cs = std::max(cs, std::min({want, kMaxCluster, std::max(1, T / kTopkMinKeys)}));
     }
   }

@@ -380,6 +380,52 @@ struct LabelSource {
   }
 };
 
+// The key of rank r (1 = largest) among the ns <= kRankCount keys of a list
+// (16-byte aligned, zero-padded to a multiple of 64; zero is below every key
+// of a non-NaN score): each key's counts of larger and equal keys, split over
+// P threads when the list is short.  Writes misc[M_THR] (the key) and
+// misc[M_NEED] (its rank among the keys equal to it).  scratch: 2*kTopkThreads
+// words.  Block-uniform; ends with a barrier.
+__device__ __forceinline__ void rank_in_list(const uint32_t* sk, int ns, uint32_t r,
+                                             uint32_t* scratch, uint32_t* misc) {
+  const int P = ns <= 64 ? 4 : (ns <= 128 ? 2 : 1);
+  const int per = kTopkThreads / P;
+  const int i = threadIdx.x % per, part = threadIdx.x / per;
+  const int span = ((ns + 63) & ~63) / P;
+  uint32_t* pgt = scratch;
+  uint32_t* peq = scratch + kTopkThreads;
+  if (i < ns) {
+    const uint32_t mine = sk[i];
+    uint32_t gt = 0u, eq = 0u;
+    const uint4* v = reinterpret_cast<const uint4*>(sk + part * span);
+    for (int j = 0; j < span / 4; j += 4) {
+      const uint4 x[4] = {v[j], v[j + 1], v[j + 2], v[j + 3]};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gt += (x[q].x > mine ? 1u : 0u) + (x[q].y > mine ? 1u : 0u) +
+              (x[q].z > mine ? 1u : 0u) + (x[q].w > mine ? 1u : 0u);
+        eq += (x[q].x == mine ? 1u : 0u) + (x[q].y == mine ? 1u : 0u) +
+              (x[q].z == mine ? 1u : 0u) + (x[q].w == mine ? 1u : 0u);
+      }
+    }
+    pgt[threadIdx.x] = gt;
+    peq[threadIdx.x] = eq;
+  }
+  __syncthreads();
+  if (threadIdx.x < ns) {
+    uint32_t gt = 0u, eq = 0u;
+    for (int q = 0; q < P; ++q) {
+      gt += pgt[q * per + threadIdx.x];
+      eq += peq[q * per + threadIdx.x];
+    }
+    if (gt < r && r <= gt + eq) {  // every thread holding the result's value
+      misc[M_THR] = sk[threadIdx.x];
+      misc[M_NEED] = r - gt;
+    }
+  }
+  __syncthreads();
+}
+
 // List select: the key of rank r (1 = largest) among the live items of a key
 // array in shared memory.  Source item i < n has key key0[i] and token tok0(i);
 // the live items are those that carry the prefix pf above bit `top` (top = 32:
@@ -509,44 +555,7 @@ __device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0
 
   uint32_t thr;
   if (st && ns <= kRankCount) {
-    // Each item's count of larger and of equal keys, split over P threads
-    // when the list is short; the list is zero-padded to a multiple of 64.
-    const int P = ns <= 64 ? 4 : (ns <= 128 ? 2 : 1);
-    const int per = kTopkThreads / P;
-    const int i = threadIdx.x % per, part = threadIdx.x / per;
-    const int span = ((ns + 63) & ~63) / P;
-    uint32_t* pgt = lists + buf * 2 * kListCap;  // the list buffer not in use
-    uint32_t* peq = pgt + kTopkThreads;
-    if (i < ns) {
-      const uint32_t mine = sk[i];
-      uint32_t gt = 0u, eq = 0u;
-      const uint4* v = reinterpret_cast<const uint4*>(sk + part * span);
-      for (int j = 0; j < span / 4; j += 4) {
-        const uint4 x[4] = {v[j], v[j + 1], v[j + 2], v[j + 3]};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          gt += (x[q].x > mine ? 1u : 0u) + (x[q].y > mine ? 1u : 0u) +
-                (x[q].z > mine ? 1u : 0u) + (x[q].w > mine ? 1u : 0u);
-          eq += (x[q].x == mine ? 1u : 0u) + (x[q].y == mine ? 1u : 0u) +
-                (x[q].z == mine ? 1u : 0u) + (x[q].w == mine ? 1u : 0u);
-        }
-      }
-      pgt[threadIdx.x] = gt;
-      peq[threadIdx.x] = eq;
-    }
-    __syncthreads();
-    if (threadIdx.x < ns) {
-      uint32_t gt = 0u, eq = 0u;
-      for (int q = 0; q < P; ++q) {
-        gt += pgt[q * per + threadIdx.x];
-        eq += peq[q * per + threadIdx.x];
-      }
-      if (gt < r && r <= gt + eq) {  // every thread holding the result's value
-        misc[M_THR] = sk[threadIdx.x];
-        misc[M_NEED] = r - gt;
-      }
-    }
-    __syncthreads();
+    rank_in_list(sk, ns, r, lists + buf * 2 * kListCap, misc);  // the list buffer not in use
     thr = misc[M_THR];
     need = misc[M_NEED];
   } else {  // every bit fixed: the live items all equal the prefix
