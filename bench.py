@@ -334,7 +334,11 @@ def time_device(step: Step, steps: int, warmup: int):
 
 def time_e2e(step: Step, steps: int, warmup: int):
     """Same step through the public API with host buffers: H2D of the query and of
-    the new token's K/V rows (into the caches at position T-1), the step, D2H of O."""
+    the new token's K/V rows (into the caches at position T-1), the step, D2H of O.
+
+    The copies and the step are captured in one CUDA graph with timing events at
+    its ends (a decode loop replays such a graph every token), so the time is the
+    GPU's, copies included, without host launch gaps."""
     import torch
 
     w = step.w
@@ -347,30 +351,41 @@ def time_e2e(step: Step, steps: int, warmup: int):
                                          ctypes.c_size_t, ctypes.c_size_t, ctypes.c_size_t,
                                          ctypes.c_int, ctypes.c_void_p]
     row = w.d * 2
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
 
-    def one():
-        e0.record()
+    def copies_and_step():
+        stream = torch.cuda.current_stream()
         step.Q.copy_(q_h, non_blocking=True)
         for src, cache in zip(kv_h, (step.K, step.V)):
             rc = cudart.cudaMemcpy2DAsync(cache.data_ptr() + (w.T - 1) * row, w.T * row,
                                           src.data_ptr(), row, row, w.B * w.Hkv, 1,
                                           stream.cuda_stream)
             assert rc == 0, rc
-        step.replay()
+        for s in step.stages():
+            s()
         o_h.copy_(step.O, non_blocking=True)
+
+    copies_and_step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        e0.record()
+        copies_and_step()
         e1.record()
+
+    def one():
+        flush_l2(step.flush)
+        g.replay()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1)
 
     for _ in range(warmup):
-        flush_l2(step.flush)
         one()
     tot = 0.0
     for _ in range(steps):
-        flush_l2(step.flush)
         tot += one()
+    del g
     h2d = q_h.numel() * 2 + 2 * kv_h[0].numel() * 2
     return tot, h2d, o_h.numel() * 4
 

@@ -15,8 +15,10 @@
 // Staging: each lane copies exactly the bytes it later reads with cp.async
 // into a per-warp ring of kAttnStages steps, so the pipeline needs neither
 // block barriers nor cross-lane hand-off: cp.async.wait_group is the only
-// wait.  Per row: 16 FMAs + 3 xor-shuffles for the logit, an online-softmax
-// update (running max m, sum l, log2 domain), 16 FMAs into the accumulator.
+// wait.  Per row: 8 paired FMAs + 3 xor-shuffles for the logit, an
+// online-softmax update (running max m, sum l, log2 domain; the accumulator
+// rescaled only when the warp meets a new maximum), 8 paired FMAs into the
+// accumulator.
 // Warps then merge through shared memory; with S > 1 each split writes
 // (m, l, unnormalised o) to the workspace and the head's last split to finish
 // (found by an arrival counter) combines them.
@@ -55,27 +57,55 @@ __device__ __forceinline__ int nb_total(const AttnParams& p) {
   return (p.T + p.block - 1) / p.block;
 }
 
-__device__ __forceinline__ float dot8(const uint4& v, const float* q) {
-  float a = bf_lo(v.x) * q[0];
-  a = fmaf(bf_hi(v.x), q[1], a);
-  a = fmaf(bf_lo(v.y), q[2], a);
-  a = fmaf(bf_hi(v.y), q[3], a);
-  a = fmaf(bf_lo(v.z), q[4], a);
-  a = fmaf(bf_hi(v.z), q[5], a);
-  a = fmaf(bf_lo(v.w), q[6], a);
-  a = fmaf(bf_hi(v.w), q[7], a);
-  return a;
+// d0 += a0*b0 and d1 += a1*b1, each rounded once: one paired fp32 FMA.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rd, {%0, %1};\n fma.rn.f32x2 rd, ra, rb, rd;\n mov.b64 {%0, %1}, rd;\n}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-__device__ __forceinline__ void axpy8(float* acc, float a, float p, const uint4& v) {
-  acc[0] = fmaf(acc[0], a, p * bf_lo(v.x));
-  acc[1] = fmaf(acc[1], a, p * bf_hi(v.x));
-  acc[2] = fmaf(acc[2], a, p * bf_lo(v.y));
-  acc[3] = fmaf(acc[3], a, p * bf_hi(v.y));
-  acc[4] = fmaf(acc[4], a, p * bf_lo(v.z));
-  acc[5] = fmaf(acc[5], a, p * bf_hi(v.z));
-  acc[6] = fmaf(acc[6], a, p * bf_lo(v.w));
-  acc[7] = fmaf(acc[7], a, p * bf_hi(v.w));
+// dot product of 8 bf16 values with 8 fp32 values: even and odd elements
+// accumulated side by side, then added
+__device__ __forceinline__ float dot8(const uint4& v, const float* q) {
+  float e = bf_lo(v.x) * q[0], o = bf_hi(v.x) * q[1];
+  fma2(e, o, bf_lo(v.y), bf_hi(v.y), q[2], q[3]);
+  fma2(e, o, bf_lo(v.z), bf_hi(v.z), q[4], q[5]);
+  fma2(e, o, bf_lo(v.w), bf_hi(v.w), q[6], q[7]);
+  return e + o;
+}
+
+// acc[0..8) += p * v (8 bf16 values)
+__device__ __forceinline__ void axpy8(float* acc, float p, const uint4& v) {
+  fma2(acc[0], acc[1], p, p, bf_lo(v.x), bf_hi(v.x));
+  fma2(acc[2], acc[3], p, p, bf_lo(v.y), bf_hi(v.y));
+  fma2(acc[4], acc[5], p, p, bf_lo(v.z), bf_hi(v.z));
+  fma2(acc[6], acc[7], p, p, bf_lo(v.w), bf_hi(v.w));
+}
+
+// One row of the online softmax for one lane: running max m and sum l (log2
+// domain) and the lane's 16 output dims acc, with the row's logit x and its V
+// chunks.  The accumulator is rescaled only when some lane of the warp meets a
+// new maximum (a warp-uniform branch, rare after the first rows).  Every lane
+// of the warp calls it; valid: the lane's row exists.
+__device__ __forceinline__ void online_row(bool valid, float x, float& m, float& l, float* acc,
+                                           const uint4& vlo, const uint4& vhi) {
+  const bool grow = valid && x > m;
+  if (__any_sync(0xffffffffu, grow)) {
+    const float a = grow ? exp2f(m - x) : 1.f;  // 0 when m is still -inf
+    if (grow) {
+      l *= a;
+      m = x;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] *= a;
+  }
+  if (valid) {
+    const float pw = exp2f(x - m);
+    l += pw;
+    axpy8(acc, pw, vlo);
+    axpy8(acc + 8, pw, vhi);
+  }
 }
 
 // weight of a partial with running max m against a common max mn (0 if empty)
@@ -200,19 +230,8 @@ k_attend(const AttnParams p) {
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 4);
     const int lr = w_begin + n * 4 + g;
-    if (lr < w_end && (!kSparse || idx_s[lr] >= 0)) {
-      float a = 1.f;
-      if (x > m) {
-        a = exp2f(m - x);  // 0 when m is still -inf
-        l *= a;
-        m = x;
-      }
-      const float pw = exp2f(x - m);
-      l += pw;
-      const uint4 vlo = st[16 + c], vhi = st[24 + c];
-      axpy8(acc, a, pw, vlo);
-      axpy8(acc + 8, a, pw, vhi);
-    }
+    const bool valid = lr < w_end && (!kSparse || idx_s[lr] >= 0);
+    online_row(valid, x, m, l, acc, st[16 + c], st[24 + c]);
   }
   cp_async_wait<0>();
 
@@ -278,13 +297,22 @@ k_attend(const AttnParams p) {
     if (last) {
       __threadfence();
       const float* all = p.partial + (size_t)bh * S * kPartialStride;
+      // the splits' (m, l) side by side in shared memory (the ring is free),
+      // each split's weight once, then every dim's weighted sum with its
+      // loads independent of one another
+      float* ms = reinterpret_cast<float*>(ring);  // [S] m, then [S] weight
+      float* wt = ms + S;
+      for (int s = j; s < S; s += kAttnThreads) ms[s] = __ldcg(all + s * kPartialStride);
+      __syncthreads();
       float Mg = -INFINITY;
-      for (int s = 0; s < S; ++s) Mg = fmaxf(Mg, __ldcg(all + s * kPartialStride));
+      for (int s = 0; s < S; ++s) Mg = fmaxf(Mg, ms[s]);
+      for (int s = j; s < S; s += kAttnThreads) wt[s] = rescale(ms[s], Mg);
+      __syncthreads();
       float Lg = 0.f, og = 0.f;
+#pragma unroll 8
       for (int s = 0; s < S; ++s) {
-        const float a = rescale(__ldcg(all + s * kPartialStride), Mg);
-        Lg = fmaf(__ldcg(all + s * kPartialStride + 1), a, Lg);
-        og = fmaf(__ldcg(all + s * kPartialStride + 4 + j), a, og);
+        Lg = fmaf(__ldcg(all + s * kPartialStride + 1), wt[s], Lg);
+        og = fmaf(__ldcg(all + s * kPartialStride + 4 + j), wt[s], og);
       }
       p.O[(size_t)bh * kHeadDim + j] = og / Lg;
       if (p.lse && j == 0) p.lse[bh] = (Mg + log2f(Lg)) * 0.69314718055994530942f;

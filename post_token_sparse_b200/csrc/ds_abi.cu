@@ -158,10 +158,14 @@ struct TopkPlan {
 // A head of at most kSample tokens is one CTA (it computes every key of the
 // head anyway).  Longer heads are cut so that one CTA's expected number of
 // candidates -- the tokens inside the sample bracket -- stays near half its
-// list, and, with few heads, further (down to kTopkMinKeys tokens per CTA) to
-// fill one wave of the cluster grid.
+// list, and, with few heads, further (down to kTopkMinKeys tokens per CTA):
+// into the largest cluster size of which every head's cluster runs at once.
 constexpr int kTopkMinKeys = 2048;
-constexpr int kTopkClusterWave = 384;
+// Clusters of each size that run at once on B200 at three selection CTAs per
+// SM (cudaOccupancyMaxActiveClusters: clusters are placed whole inside a GPC,
+// so large clusters pack worse).  Spreading uses these sizes only.
+constexpr int kSpreadSizes[] = {16, 14, 12, 10, 8, 6, 4, 2};
+constexpr int kActiveClusters[] = {21, 24, 31, 41, 48, 71, 104, 222};
 
 bool plan_topk(int BH, int T, int k, TopkPlan* out) {
   int cs = (T + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
@@ -171,12 +175,12 @@ bool plan_topk(int BH, int T, int k, TopkPlan* out) {
     const double frac = 2.0 * (kBracketSigmas * std::sqrt(e * (1.0 - p)) + 3.0) / kSample;
     const double max_chunk = 0.5 * kCandCap / std::max(frac, 1e-9);
     cs = std::max(cs, (int)std::min<double>(kMaxCluster, std::ceil(T / max_chunk)));
-    // few heads: spread each over more CTAs, up to one wave.  Clusters are
-    // placed whole inside a GPC, so at three selection CTAs per SM about 384
-    // CTAs of clusters run at once; a second wave would double the time.
-    if (BH * cs < kTopkClusterWave) {
-      const int want = std::max(1, kTopkClusterWave / BH);
-      cs = std::max(cs, std::min({want, kMaxCluster, std::max(1, T / kTopkMinKeys)}));
+    for (int i = 0; i < 8; ++i) {
+      const int c = kSpreadSizes[i];
+      if (c > cs && c <= T / kTopkMinKeys && BH <= kActiveClusters[i]) {
+        cs = c;
+        break;
+      }
     }
   }
   int chunk = (T + cs - 1) / cs;

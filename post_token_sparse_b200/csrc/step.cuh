@@ -119,19 +119,7 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 4);
-    if (w_begin + s * 4 + g < w_end) {
-      float a = 1.f;
-      if (x > m) {
-        a = exp2f(m - x);
-        l *= a;
-        m = x;
-      }
-      const float pw = exp2f(x - m);
-      l += pw;
-      const uint4 vlo = st[16 + c], vhi = st[24 + c];
-      axpy8(acc, a, pw, vlo);
-      axpy8(acc + 8, a, pw, vhi);
-    }
+    online_row(w_begin + s * 4 + g < w_end, x, m, l, acc, st[16 + c], st[24 + c]);
   }
   cp_async_wait<0>();
 #pragma unroll

@@ -817,26 +817,31 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
         top >= 32 ? 0u : lo >> top, krem, 0, -1, 0u, 0u, hist, lists, misc, gtm, eqm, c0, len,
         need);
   } else if (lo != hi) {
+    // a cluster: radix select over the candidates with histograms merged over
+    // the cluster, starting at the highest bit where lo and hi differ (every
+    // candidate shares the bits above it)
     const uint32_t ncand = misc[M_NCAND];
-    uint32_t p = 0, r = krem;
-    for (int d = 0; d < 3; ++d) {
-      const int nb = digit_bins(d);
-      uint32_t* mg = sm + (d == 1 ? L.merged1 : L.merged0);
+    int t = 32 - __clz(lo ^ hi);
+    uint32_t p = t >= 32 ? 0u : lo >> t, r = krem;
+    for (int round = 0; t > 0; ++round) {
+      const int bits = t < 11 ? t : 11;
+      const int sh = t - bits;
+      const int nb = 1 << bits;
+      uint32_t* mg = sm + ((round & 1) ? L.merged1 : L.merged0);
       for (int i = threadIdx.x; i < nb; i += kTopkThreads) hist[i] = 0u;
-      if (cs > 1)
-        for (int i = threadIdx.x; i < nb; i += kTopkThreads) mg[i] = 0u;
+      for (int i = threadIdx.x; i < nb; i += kTopkThreads) mg[i] = 0u;
       cluster_or_cta_sync(cs);
-      const int hs = d > 0 ? digit_shift(d - 1) : 0;
       for (uint32_t s = threadIdx.x; s < ncand; s += kTopkThreads) {
         const uint32_t key = cand_key[s];
-        if (d == 0 || (key >> hs) == p) atomicAdd(&hist[(key >> digit_shift(d)) & (nb - 1)], 1u);
+        if (t >= 32 || (key >> t) == p) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
       }
       __syncthreads();
       const uint32_t* h = cluster_hist(hist, mg, nb, cs);
       find_bin(h, nb, r, misc + 48, misc + M_BIN);
-      p = (p << digit_bits(d)) | misc[M_BIN];
+      p = (p << bits) | misc[M_BIN];
       r -= misc[M_ABOVE];
       __syncthreads();
+      t = sh;
     }
     need = r;
     for (uint32_t s = threadIdx.x; s < ncand; s += kTopkThreads) {
