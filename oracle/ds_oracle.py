@@ -75,6 +75,25 @@ model to tune a threshold on, the reading taken is:
                are every token of those blocks (clipped to T), ascending
   attention    as above, over the kept tokens
 
+Hierarchical top-k (page "A Training-free Sub-quadratic Cost Transformer
+Model Serving Framework With Hierarchically Pruned Attention", Core idea:
+attention locality, nearby tokens score alike; Technical framework: a
+hierarchy of tokens searched tree-like for each query's important keys).  The
+page leaves the hierarchy and the search open (its examples, k-means and
+binary search, are the summary's guesses); the reading taken here is a
+binary hierarchy of contiguous ranges searched top-down:
+
+  start        k parts of [0, T): part i is [floor(iT/k), floor((i+1)T/k))
+  level        every part of more than one token is halved (the first half
+               takes the extra token); each part is scored by the approximate
+               score of its first token; the k best parts stay (score
+               descending, start ascending)
+  end          after ceil(log2 of the longest start part) levels every part
+               is one token: the k kept tokens, ascending
+
+It reads about 2k·log2(T/k) label rows instead of T, and equals the exact
+top-k when the search is exhaustive (k = T) or the scores fall with position.
+
 Pins (see tests/test_oracle_pins.py): bf16 decoding against known bit
 patterns; label gather against the identity/permutation cases and a
 per-element brute force; score against one-hot queries and the attention
@@ -98,6 +117,7 @@ __all__ = [
     "calibrate_importance", "calibrate_select", "calibrate",
     "group_score", "group_attend", "group_sparse_step",
     "block_score", "block_tokens", "block_sparse_step",
+    "hier_topk_head", "hier_topk",
 ]
 
 
@@ -396,3 +416,35 @@ def block_sparse_step(Q, K, V, C, bs, kb, scale):
             toks = block_tokens(bidx[b, h], bs, T)
             O[b, h], L[b, h], _ = attend_head(Q[b, h], K[b, g], V[b, g], toks, scale)
     return {"s32": s32, "sb": sb, "bidx": bidx, "O": O, "lse": L}
+
+
+# ---- hierarchical top-k ------------------------------------------------------------
+
+def hier_topk_head(s: np.ndarray, k: int) -> np.ndarray:
+    """The k tokens the top-down search over contiguous ranges keeps (ascending)."""
+    s = np.asarray(s)
+    T = s.shape[0]
+    if not 1 <= k <= T:
+        raise ValueError("need 1 <= k <= T")
+    parts = [((i * T) // k, ((i + 1) * T) // k) for i in range(k)]
+    while any(e - b > 1 for b, e in parts):
+        children = []
+        for b, e in parts:
+            if e - b > 1:
+                m = b + (e - b + 1) // 2
+                children += [(b, m), (m, e)]
+            else:
+                children.append((b, e))
+        children.sort(key=lambda c: (-s[c[0]], c[0]))  # first token's score, then start
+        parts = sorted(children[:k])
+    return np.array([b for b, _ in parts], np.int32)
+
+
+def hier_topk(s: np.ndarray, k: int) -> np.ndarray:
+    """idx [..., k] int32 for scores [..., T]."""
+    lead = s.shape[:-1]
+    flat = s.reshape(-1, s.shape[-1])
+    out = np.empty((flat.shape[0], k), np.int32)
+    for i in range(flat.shape[0]):
+        out[i] = hier_topk_head(flat[i], k)
+    return out.reshape(*lead, k)

@@ -28,6 +28,10 @@ What pins what:
                       last block; bs = 1 is top-k of the clamped scores;
                       blocks' tokens contiguous and clipped; the step equals
                       attention over the blocks' tokens
+  hierarchical top-k  the hand-derived worked example (tests/golden/
+                      hier_worked.json, odd lengths included); k = T and
+                      scores falling with position and constant scores
+                      give the exact top-k
   calibration         brute-force mean over (query, token) pairs; the
                       query-head -> KV-head map on marked KV heads; ties to
                       the lower channel; channel-permutation equivariance;
@@ -501,8 +505,35 @@ def pin_block_tokens_and_step(orc):
     assert np.array_equal(one["bidx"], orc.topk(np.maximum(one["s32"], 0), 5))
 
 
+# ---------------------------------------------------------------------------
+# hierarchical top-k
+
+def pin_hier_topk(orc):
+    g = _load("hier_worked.json")
+    s = np.array(g["scores"])
+    for k, want in g["expected"].items():
+        assert list(orc.hier_topk_head(s, int(k))) == want, (k, orc.hier_topk_head(s, int(k)))
+    for case in ("odd", "uneven"):
+        assert list(orc.hier_topk_head(np.array(g[case]["scores"]), g[case]["k"])) == \
+            g[case]["expected"], case
+    rng = np.random.default_rng(71)
+    for T, k in [(1, 1), (13, 13), (64, 5), (100, 7), (257, 16)]:
+        x = rng.standard_normal(T)
+        # exhaustive search (k = T): every token
+        if k == T:
+            assert list(orc.hier_topk_head(x, k)) == list(range(T))
+        # scores falling with position: each part's first token is its best
+        dec = -np.arange(T, dtype=np.float64) + 0.01 * (T - np.arange(T)) ** 0.5
+        assert list(orc.hier_topk_head(dec, k)) == list(range(k))
+        # all equal: ties to the lower start narrow onto the first k tokens, the
+        # exact top-k's answer too
+        assert list(orc.hier_topk_head(np.zeros(T), k)) == list(range(k))
+        got = orc.hier_topk_head(x, k)
+        assert len(set(got)) == k and all(0 <= t < T for t in got) and list(got) == sorted(got)
+
+
 PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
         pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding,
         pin_calib_bruteforce, pin_calib_groups_and_order, pin_calib_permutation,
         pin_calib_recovers_outliers, pin_group_score, pin_group_step, pin_block_score,
-        pin_block_tokens_and_step]
+        pin_block_tokens_and_step, pin_hier_topk]

@@ -88,6 +88,15 @@ MUTATIONS = [
     ("block tokens not clipped", "for t in range(j * bs, min((j + 1) * bs, T))]",
      "for t in range((j * bs), (j + 1) * bs)]"),
     ("block step selects on tokens, not blocks", "bidx = topk(sb, kb)", "bidx = topk(s32, kb)"),
+    ("hierarchy halves the other way", "m = b + (e - b + 1) // 2", "m = b + (e - b) // 2"),
+    ("hierarchy scores parts by their last token",
+     "children.sort(key=lambda c: (-s[c[0]], c[0]))", "children.sort(key=lambda c: (-s[c[1] - 1], c[0]))"),
+    ("hierarchy ties to the higher start",
+     "children.sort(key=lambda c: (-s[c[0]], c[0]))", "children.sort(key=lambda c: (-s[c[0]], -c[0]))"),
+    ("hierarchy keeps the worst parts",
+     "children.sort(key=lambda c: (-s[c[0]], c[0]))", "children.sort(key=lambda c: (s[c[0]], c[0]))"),
+    ("hierarchy starts from unequal parts", "parts = [((i * T) // k, ((i + 1) * T) // k) for i in range(k)]",
+     "parts = [(i * (T // k), (i + 1) * (T // k) if i < k - 1 else T) for i in range(k)]"),
 ]
 
 
