@@ -631,6 +631,78 @@ def block_entry(w, inputs, hbm_peak, bs: int = 64, steps: int = 50):
             "tokens_heads_per_s": w.B * w.Hq * w.T / (ms * 1e-3)}
 
 
+def offload_entry(w, hbm_peak):
+    """KV offload: K and V of the workload in page-locked host memory, the label
+    cache on the GPU.  A step (new label row, score + top-k, sparse attention)
+    reads over the host link only the kept K/V rows; dense decode reads all."""
+    import numpy as np
+    import torch
+
+    import post_token_sparse_b200 as ds
+
+    Qb, Kb, Vb = dsgen.qkv(w)
+    Q = torch.from_numpy(Qb.view(np.int16)).view(torch.bfloat16).cuda()
+    K = torch.from_numpy(Kb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    del Kb
+    V = torch.from_numpy(Vb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    del Vb
+    C = torch.from_numpy(dsgen.channels(w)).cuda()
+    label = torch.empty((w.B, w.Hq, w.T, w.r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(K, C, label, 0, w.T)  # the prompt (setup)
+    BH = w.B * w.Hq
+    idx = torch.empty((BH, w.k), dtype=torch.int32, device="cuda")
+    O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    dims = ds.dims_of(Q, K, w.r)
+    ws = ds.workspace(ds.OP_SPARSE_DECODE, dims, w.T, w.k, "cuda")
+    wsd = ds.workspace(ds.OP_DECODE, dims, w.T, w.T, "cuda")
+
+    def step():
+        ds.label_append(K, C, label, w.T - 1, 1)
+        ds.score_topk(Q, C, label, idx, w.T)
+        ds.sparse_decode(Q, K, V, idx, O, w.T, w.scale, ws=ws)
+
+    ms = time_graph(step, 5, 2)
+    msd = time_graph(lambda: ds.decode(Q, K, V, O, w.T, w.scale, ws=wsd), 2, 1)
+    link = w.B * w.Hq * w.k * 2 * w.d * 2 + w.B * w.Hkv * w.d * 2
+    del K, V
+    return {"us_per_step": ms * 1e3, "host_link_bytes_per_step": link,
+            "host_link_gbs": link / (ms * 1e-3) / 1e9, "dense_us_per_step": msd * 1e3,
+            "dense_host_link_bytes": w.dense_bytes(), "speedup_vs_dense": msd / ms}
+
+
+def hier_entry(w, inputs, hbm_peak, steps: int = 50):
+    """Hierarchical (top-down) selection in place of the exact top-k: the step's
+    label append, ds_hier_score_topk and ds_sparse_decode over its k tokens."""
+    import math
+
+    import torch
+
+    import post_token_sparse_b200 as ds
+
+    Q, K, V = inputs
+    C = torch.from_numpy(dsgen.channels(w)).cuda()
+    label = torch.empty((w.B, w.Hq, w.T, w.r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(K, C, label, 0, w.T)
+    BH = w.B * w.Hq
+    idx = torch.empty((BH, w.k), dtype=torch.int32, device="cuda")
+    O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    ws = ds.workspace(ds.OP_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
+
+    def step():
+        ds.label_append(K, C, label, w.T - 1, 1)
+        ds.hier_score_topk(Q, C, label, idx, w.T)
+        ds.sparse_decode(Q, K, V, idx, O, w.T, w.scale, ws=ws)
+
+    ms = time_graph(step, steps, 3)
+    levels = max(0, math.ceil(math.log2(-(-w.T // w.k)))) if w.T > w.k else 0
+    rows = 2 * w.k * levels
+    nb = BH * (rows * w.r * 2 + w.k * (2 * w.d * 2 + 4) + w.d * 6)
+    return {"us_per_step": ms * 1e3, "levels": levels, "label_rows_read_per_head": rows,
+            "bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": nb / (ms * 1e-3) / 1e9 / hbm_peak,
+            "tokens_heads_per_s": BH * w.T / (ms * 1e-3)}
+
+
 def _rounded(e):
     return {k: (_rounded(v) if isinstance(v, dict) else round(v, 4) if isinstance(v, float)
                 else v) for k, v in e.items()}
@@ -664,6 +736,10 @@ def run_sweep(skip: str, hbm_peak: float):
             e["group_shared"] = group_entry(ww, inp, hbm_peak)
         if first_of_set and ww.T >= 16384:
             e["block_select"] = block_entry(ww, inp, hbm_peak, steps=20)
+        if ww.T >= 262144:
+            e["kv_offload"] = offload_entry(ww, hbm_peak)
+        if ww.k <= 2048 and (first_of_set or ww.Hq > ww.Hkv) and ww.T > 4096:
+            e["hier_select"] = hier_entry(ww, inp, hbm_peak, steps=20)
         out[name] = _rounded(e)
         if name == dsgen.ORDER[-1] and name.startswith("sweep"):
             full = ww.with_(name="sweep-B32-H32-T32K-r128-kT", r=ww.d, k=ww.T)
@@ -768,6 +844,7 @@ def main():
         line["cpu_baseline"] = time_oracle(base, args.cpu_seconds)
         line["calibrate"] = _rounded(calib_entry(w, inputs[1], hbm_peak))
         line["block_select"] = _rounded(block_entry(w, inputs, hbm_peak))
+        line["hier_select"] = _rounded(hier_entry(w, inputs, hbm_peak))
     del inputs
     torch.cuda.empty_cache()
     if rank == 0 and world == 1:

@@ -33,6 +33,13 @@
  *   - All data pointers are DEVICE pointers owned by the caller; the library
  *     never allocates, frees or synchronises.  Every pointer must be 16-byte
  *     aligned.  Calls are asynchronous on `stream` (0 = legacy default).
+ *   - KV offload: K and V may instead be page-locked host memory mapped into
+ *     the device's address space (cudaHostAlloc, or pinned memory under
+ *     unified addressing).  The kernels then read over the host link only the
+ *     rows they use: the kept rows in the sparse calls, one row per step in
+ *     ds_label_append (Double Sparsity page, Abstract and Experimental
+ *     highlights: combined with offloading the KV cache to host memory).
+ *     Other host memory is refused with DS_ERR_INVALID_ARG before launch.
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns DS_ERR_INVALID_ARG (or DS_ERR_UNSUPPORTED for a valid
  *     but unimplemented shape) and launches nothing.
@@ -314,6 +321,29 @@ ds_status ds_block_sparse_decode(const void* Q, const void* K, const void* V,
                                  const int32_t* bidx, float* O, float* lse, ds_dims dims,
                                  int32_t T, int32_t bs, int32_t kb, float scale, void* ws,
                                  size_t ws_bytes, ds_stream_t stream);
+
+/*
+ * ds_hier_score_topk -- hierarchical (top-down) token selection.
+ *
+ * Page "A Training-free Sub-quadratic Cost Transformer Model Serving
+ * Framework With Hierarchically Pruned Attention": nearby tokens score alike
+ * (Core idea, attention locality), and a hierarchy of tokens is searched
+ * tree-like for each query's important keys (Technical framework).  Reading:
+ * k contiguous parts of [0, T) (part i = [floor(iT/k), floor((i+1)T/k))) are
+ * halved level by level (the first half takes the extra token); each part is
+ * scored by its first token's approximate score (as ds_score computes it); the
+ * k best parts stay (score descending, start ascending); when every part is
+ * one token, idx[bh] = those k tokens, ascending.  Reads about 2k*log2(T/k)
+ * label rows per head instead of T; equals ds_score_topk when the scores fall
+ * with position or k = T, and otherwise is an approximation that relies on
+ * locality.
+ *
+ * Q, C, label as for ds_score.  idx: [B*Hq, k] int32.  Requires r in
+ * {8,16,32,64,128}, 1 <= k <= min(T, 2048), T <= T_cap.  One launch, no
+ * workspace.
+ */
+ds_status ds_hier_score_topk(const void* Q, const int32_t* C, const void* label, int32_t* idx,
+                             ds_dims dims, int32_t T, int32_t k, ds_stream_t stream);
 
 /*
  * ds_calibrate -- offline channel calibration: the label channels C.

@@ -76,6 +76,7 @@ def _load():
         "ds_calibrate": [vp, i32, vp, Dims, i32, vp, vp, vp, ctypes.c_size_t, vp],
         "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
+        "ds_hier_score_topk": [vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_block_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, i32, ctypes.c_float,
                                    vp, ctypes.c_size_t, vp],
         "ds_group_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, vp,
@@ -115,8 +116,10 @@ def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
         return None
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
+    # K and V may also be pinned host tensors (KV offload; see include/ds.h)
+    if not t.is_cuda and not (name in ("K", "V") and t.is_pinned()):
+        raise TypeError(f"{name} must be a CUDA tensor" +
+                        (" or a pinned host tensor" if name in ("K", "V") else ""))
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -162,7 +165,7 @@ def label_append(K, C, label, t0: int, n: int):
     dims = Dims(B, Hq, Hkv, d, T_cap, r)
     _check(_lib.ds_label_append(_ptr(K, torch.bfloat16, "K"), _ptr(C, torch.int32, "C"),
                                 _ptr(label, torch.bfloat16, "label"), dims, t0, n,
-                                _stream(K.device)), "ds_label_append")
+                                _stream(label.device)), "ds_label_append")
 
 
 def score(Q, C, label, scores, T: int):
@@ -286,6 +289,16 @@ def block_sparse_decode(Q, K, V, bidx, O, T: int, bs: int, scale: float, lse=Non
                                        _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"),
                                        dims, T, bs, kb, scale, _ptr(ws, None, "ws"), nbytes,
                                        _stream(Q.device)), "ds_block_sparse_decode")
+
+
+def hier_score_topk(Q, C, label, idx, T: int):
+    """Hierarchical (top-down) selection of k = idx.shape[-1] tokens per head."""
+    B, Hq, T_cap, r = label.shape
+    dims = Dims(B, Hq, Hq, Q.shape[-1], T_cap, r)
+    _check(_lib.ds_hier_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
+                                   _ptr(label, torch.bfloat16, "label"),
+                                   _ptr(idx, torch.int32, "idx"), dims, T, idx.shape[-1],
+                                   _stream(Q.device)), "ds_hier_score_topk")
 
 
 def calibrate(Qc, K, C, T: int, importance=None, ws=None):

@@ -30,6 +30,27 @@ thread_local char g_cuda_err[256] = "no error";
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// K and V may be device memory or page-locked host memory mapped into the
+// device's address space (the KV cache offloaded to the host; kernels then
+// read the rows they need over the host link).  Any other host memory is
+// refused before a launch could touch it.  When the runtime cannot be asked
+// (no device), the launch itself reports the error.
+ds_status check_kv_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return DS_OK;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return DS_OK;
+  if (a.type == cudaMemoryTypeHost && a.devicePointer == p) return DS_OK;
+  return DS_ERR_INVALID_ARG;
+}
+
+ds_status check_kv(const void* K, const void* V) {
+  ds_status s = check_kv_ptr(K);
+  return s != DS_OK || V == nullptr ? s : check_kv_ptr(V);
+}
+
 ds_status cuda_fail(cudaError_t e) {
   std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e),
                 cudaGetErrorString(e));
@@ -138,6 +159,12 @@ ds_status ensure_attrs() {
     acc(topk_attrs<LabelSource<32>>());
     acc(topk_attrs<LabelSource<64>>());
     acc(topk_attrs<LabelSource<128>>());
+    const size_t hier_max = HierLayout(TopkLayout(2 * kHierMaxK, 1)).bytes();
+    acc(allow_smem(k_hier_topk<LabelSource<8>>, hier_max));
+    acc(allow_smem(k_hier_topk<LabelSource<16>>, hier_max));
+    acc(allow_smem(k_hier_topk<LabelSource<32>>, hier_max));
+    acc(allow_smem(k_hier_topk<LabelSource<64>>, hier_max));
+    acc(allow_smem(k_hier_topk<LabelSource<128>>, hier_max));
     const size_t step_max = 227 * 1024;
     acc(allow_smem(k_step<8>, step_max));
     acc(allow_smem(k_step<16>, step_max));
@@ -420,6 +447,8 @@ ds_status ds_label_append(const void* K, const int32_t* C, void* label, ds_dims 
   const int G = dims.Hq / dims.Hkv;
   const size_t cs_bytes = (size_t)G * dims.r * sizeof(int32_t);
   if (cs_bytes > 40 * 1024) return DS_ERR_UNSUPPORTED;
+  s = check_kv(K, nullptr);
+  if (s != DS_OK) return s;
   dim3 grid((n + kLabelTile - 1) / kLabelTile, dims.B * dims.Hkv);
   k_label_append<<<grid, kLabelThreads, cs_bytes, stream>>>(
       static_cast<const uint16_t*>(K), C, static_cast<uint16_t*>(label), dims.Hq, dims.Hkv,
@@ -496,6 +525,8 @@ ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const in
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
   s = check_attend_ws(dims, k, true, ws, ws_bytes);
   if (s != DS_OK) return s;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
@@ -511,6 +542,8 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
   s = check_attend_ws(dims, T, false, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = check_kv(K, V);
   if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
@@ -562,6 +595,8 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
   const size_t need = partial_bytes(BH, sp);
   if (need > DS_NOALLOC_SCRATCH_BYTES) return DS_ERR_WORKSPACE;
   if (sp.S > 65535) return DS_ERR_UNSUPPORTED;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   void* scratch = nullptr;
@@ -602,6 +637,8 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
                      dims.r == 128;
     if (!vec) return DS_ERR_UNSUPPORTED;  // the fused score+select needs a vector path
   }
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   if (fused) {
@@ -655,6 +692,8 @@ extern "C" ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_
   if (nck > 65535 || ncq > 65535) return DS_ERR_UNSUPPORTED;
   const size_t need = ds_workspace_size(DS_OP_CALIBRATE, dims, T, Nq);
   if (!ws || ws_bytes < need || !aligned16(ws)) return DS_ERR_WORKSPACE;
+  s = check_kv(K, nullptr);
+  if (s != DS_OK) return s;
   float* pk = static_cast<float*>(ws);
   float* pq = pk + (size_t)dims.B * dims.Hkv * nck * kHeadDim;
   if ((int64_t)dims.B * (dims.Hkv + dims.Hq) > 65535) return DS_ERR_UNSUPPORTED;
@@ -726,6 +765,8 @@ extern "C" ds_status ds_group_sparse_decode(const void* Q, const void* K, const 
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
   s = check_attend_ws(dims, k, true, ws, ws_bytes);
   if (s != DS_OK) return s;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream, true);
@@ -791,7 +832,47 @@ extern "C" ds_status ds_block_sparse_decode(const void* Q, const void* K, const 
   const int rows = kb * bs;
   s = check_attend_ws(dims, rows, true, ws, ws_bytes);
   if (s != DS_OK) return s;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, bidx, O, lse, T, rows, scale, ws, stream, false, bs);
+}
+
+namespace {
+
+template <int R>
+ds_status launch_hier(const uint16_t* Q, const int32_t* C, const uint16_t* label, int32_t* idx,
+                      const ds_dims& d, int T, int k, cudaStream_t st) {
+  const size_t smem = HierLayout(TopkLayout((2 * k + 31) & ~31, 1)).bytes();
+  LabelSource<R> src{Q, C, label, nullptr, d.Hq, d.T_cap};
+  k_hier_topk<LabelSource<R>><<<d.B * d.Hq, kTopkThreads, smem, st>>>(src, idx, T, k);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" ds_status ds_hier_score_topk(const void* Q, const int32_t* C, const void* label,
+                                        int32_t* idx, ds_dims dims, int32_t T, int32_t k,
+                                        ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !C || !label || !idx || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
+      !aligned16(idx))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (k > kHierMaxK) return DS_ERR_UNSUPPORTED;
+  if (!(dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 || dims.r == 128))
+    return DS_ERR_UNSUPPORTED;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  auto Qb = static_cast<const uint16_t*>(Q);
+  auto Lb = static_cast<const uint16_t*>(label);
+  switch (dims.r) {
+    case 8: return launch_hier<8>(Qb, C, Lb, idx, dims, T, k, stream);
+    case 16: return launch_hier<16>(Qb, C, Lb, idx, dims, T, k, stream);
+    case 32: return launch_hier<32>(Qb, C, Lb, idx, dims, T, k, stream);
+    case 64: return launch_hier<64>(Qb, C, Lb, idx, dims, T, k, stream);
+    default: return launch_hier<128>(Qb, C, Lb, idx, dims, T, k, stream);
+  }
 }

@@ -202,7 +202,9 @@ k_step(const StepParams p, int chunk) {
   }
 
   // 2. selection (its first barrier publishes qs and the new row)
-  LabelSource<R> src{p.Q, p.C, p.label, nullptr, p.Hq, p.T_cap};
+  // eight label loads in flight per thread (the selection CTAs of k_topk,
+  // three per SM, keep four)
+  LabelSource<R, 8> src{p.Q, p.C, p.label, nullptr, p.Hq, p.T_cap};
   if (p.append) {
     src.over_t = p.T - 1;
     src.over_row = reinterpret_cast<const uint4*>(over16);

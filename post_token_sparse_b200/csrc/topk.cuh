@@ -327,7 +327,7 @@ struct ScoresSource {
 // are computed exactly as k_score_vec computes them (same order of fp32
 // operations), r/8 lanes per row so that every warp load reads 512 contiguous
 // bytes, with the next slice's loads in flight while a slice is consumed.
-template <int R>
+template <int R, int kSlotsT = 4>
 struct LabelSource {
   const uint16_t* Q;
   const int32_t* C;
@@ -339,7 +339,7 @@ struct LabelSource {
                                     // by the same kernel)
   static constexpr int kLanes = R / 8;
   static constexpr int kRowsPerInstr = 32 / kLanes;
-  static constexpr int kSlots = 4;
+  static constexpr int kSlots = kSlotsT;  // 16-byte loads in flight per thread
   static constexpr int kStep = kTopkWarps * kSlots * kRowsPerInstr;  // items per slice
 
   __device__ __forceinline__ void prepare(int bh, float* qs) const {
@@ -950,6 +950,143 @@ k_topk(Source src, int32_t* __restrict__ idx, int T, int k, int chunk) {
   extern __shared__ __align__(16) uint32_t sm[];
   topk_body(src, sm, (int)gridDim.x, (int)blockIdx.x, (int)blockIdx.y, T, k, chunk,
             idx + (size_t)blockIdx.y * k, nullptr);
+}
+
+}  // namespace ds
+
+namespace ds {
+
+// ---- hierarchical top-k ------------------------------------------------------
+// Page "A Training-free Sub-quadratic Cost Transformer Model Serving Framework
+// With Hierarchically Pruned Attention" (Core idea: attention locality, nearby
+// tokens score alike; Technical framework: a hierarchy of tokens searched
+// tree-like for each query's important keys).  Reading: k contiguous parts of
+// [0, T) are halved level by level (the first half takes the extra token);
+// each part is scored by its first token's approximate score; the k best parts
+// stay (score descending, start ascending); after the last level the k parts
+// are single tokens.  One CTA per head: each level scores its 2k children from
+// the label cache (one row each, LabelSource), selects k of them with the list
+// select (ties in child order = start order), and compacts the kept children
+// into the next level's parts.  About 2k*log2(T/k) label rows are read instead
+// of T.
+constexpr int kHierMaxK = 2048;
+
+struct HierLayout {
+  int nodes0, nodes1, words;  // part starts and ends, two buffers of kHierMaxK each
+  __host__ __device__ explicit HierLayout(const TopkLayout& L) {
+    nodes0 = L.words;
+    nodes1 = nodes0 + 2 * kHierMaxK;
+    words = nodes1 + 2 * kHierMaxK;
+  }
+  __host__ __device__ size_t bytes() const { return (size_t)words * 4; }
+};
+
+// grid (BH), block kTopkThreads; shared memory HierLayout(TopkLayout(2k rounded
+// up to 32, 1)).  idx: [BH, k] out, ascending.
+template <class Source>
+__global__ void __launch_bounds__(kTopkThreads, 2)
+k_hier_topk(Source src, int32_t* __restrict__ idx, int T, int k) {
+  extern __shared__ __align__(16) uint32_t sm[];
+  const int n = 2 * k;  // children per level
+  const int chunk = (n + 31) & ~31;
+  const TopkLayout L(chunk, 1);
+  const HierLayout H(L);
+  const int bh = blockIdx.x;
+  uint32_t* hist = sm;
+  uint32_t* misc = sm + L.small;
+  float* qs = reinterpret_cast<float*>(misc + 64);
+  uint32_t* gtm = sm + L.masks;
+  uint32_t* eqm = gtm + chunk / 32;
+  uint32_t* keys = sm + L.X;
+  uint32_t* lists = sm + L.lists;
+  int32_t* ps = reinterpret_cast<int32_t*>(sm + H.nodes0);  // part starts
+  int32_t* pe = ps + kHierMaxK;                               // part ends
+  int32_t* qs2 = reinterpret_cast<int32_t*>(sm + H.nodes1);
+  int32_t* qe2 = qs2 + kHierMaxK;
+
+  for (int i = threadIdx.x; i < L.small + 64; i += kTopkThreads) sm[i] = 0u;
+  for (int i = threadIdx.x; i < k; i += kTopkThreads) {
+    ps[i] = (int)(((long long)i * T) / k);
+    pe[i] = (int)(((long long)(i + 1) * T) / k);
+  }
+  src.prepare(bh, qs);
+  __syncthreads();
+
+  int maxlen = (T + k - 1) / k;
+  const int groups = chunk / 32;
+  while (maxlen > 1) {
+    // child j of part j/2: the first or second half, or nothing (a part of one
+    // token has one child)
+    auto child = [&](int j, int& b, int& e) {
+      const int i = j >> 1;
+      const int pb = ps[i], pe_ = pe[i];
+      if (pe_ - pb > 1) {
+        const int m = pb + (pe_ - pb + 1) / 2;
+        b = (j & 1) ? m : pb;
+        e = (j & 1) ? pe_ : m;
+      } else {
+        b = pb;
+        e = (j & 1) ? pb : pe_;  // empty second child
+      }
+    };
+    src.stream(bh, T, n,
+               [&](int j) {
+                 int b, e;
+                 child(j, b, e);
+                 return b;
+               },
+               [&](bool v, int j, uint32_t key, float) {
+                 if (v) {
+                   int b, e;
+                   child(j, b, e);
+                   keys[j] = e > b ? key : 0u;  // zero: below every key of a non-NaN score
+                 }
+               },
+               qs);
+    for (int i = threadIdx.x; i < 2 * groups; i += kTopkThreads) gtm[i] = 0u;
+    __syncthreads();
+    uint32_t need;
+    list_select<true, true>(keys, [](int i) { return i; }, n, 32, 0u, (uint32_t)k, 0, -1, 0u,
+                            0u, hist, lists, misc, gtm, eqm, 0, n, need);
+    // kept children in child order: all above the threshold, and the first
+    // `need` equal to it
+    uint32_t ne = 0u, ng = 0u, gm = 0u, em = 0u;
+    if (threadIdx.x < groups) {
+      gm = gtm[threadIdx.x];
+      em = eqm[threadIdx.x];
+      ne = __popc(em);
+    }
+    const uint32_t tie = block_exclusive_scan(ne, misc + 48);
+    __syncthreads();
+    uint32_t sel = gm;
+    if (threadIdx.x < groups && need > tie) {
+      const uint32_t take = min(need - tie, ne);
+      uint32_t rest = em;
+      for (uint32_t t = 0; t < take; ++t) rest &= rest - 1u;
+      sel |= em ^ rest;
+    }
+    ng = __popc(sel);
+    uint32_t pos = block_exclusive_scan(ng, misc + 48);
+    while (sel) {
+      const int bit = __ffs(sel) - 1;
+      sel &= sel - 1u;
+      int b, e;
+      child(threadIdx.x * 32 + bit, b, e);
+      if (pos < (uint32_t)k) {
+        qs2[pos] = b;
+        qe2[pos] = e;
+      }
+      ++pos;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < k; i += kTopkThreads) {
+      ps[i] = qs2[i];
+      pe[i] = qe2[i];
+    }
+    __syncthreads();
+    maxlen = (maxlen + 1) / 2;
+  }
+  for (int i = threadIdx.x; i < k; i += kTopkThreads) idx[(size_t)bh * k + i] = ps[i];
 }
 
 }  // namespace ds

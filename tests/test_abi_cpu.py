@@ -211,6 +211,18 @@ def test_block_calls_validation():
                                       NUL) == ds.DS_ERR_WORKSPACE
 
 
+def test_hier_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=5000, r=16)
+    assert lib.ds_hier_score_topk(P, P, P, P, d, 5000, 2049, NUL) == ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_hier_score_topk(P, P, P, P, d, 100, 101, NUL) == bad
+    assert lib.ds_hier_score_topk(P, P, P, P, d, 5001, 10, NUL) == bad
+    assert lib.ds_hier_score_topk(P, P, P, P, d, 100, 0, NUL) == bad
+    assert lib.ds_hier_score_topk(P, P, NUL, P, d, 100, 10, NUL) == bad
+    assert lib.ds_hier_score_topk(P, P, P, P, _dims(r=12), 100, 10, NUL) == ds.DS_ERR_UNSUPPORTED
+
+
 def test_calibrate_validation_and_workspace():
     lib = ds.lib()
     d = _dims(B=2, Hq=8, Hkv=2, T_cap=5000, r=16)
