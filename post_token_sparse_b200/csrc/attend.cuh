@@ -142,11 +142,19 @@ k_attend(const AttnParams p) {
   const uint4* qrow = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim);
   const uint4 qa = qrow[c], qb = qrow[8 + c];
 
+  // rows of this warp: [w_begin, w_end) relative to r0
+  const int rpw = ((nrows + kAttnWarps - 1) / kAttnWarps + 3) & ~3;
+  const int w_begin = min(warp * rpw, nrows);
+  const int w_end = min(w_begin + rpw, nrows);
+  const int nsteps = (w_end - w_begin + 3) >> 2;
+
   if constexpr (kSparse) {
+    // each warp stages the token ids of its own rows (no block barrier: a warp
+    // starts its gathers as soon as its own ids are in)
     if (p.block) {
       const int nb = p.rows / p.block;
       const int32_t* src = p.idx + (size_t)bh * nb;
-      for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
+      for (int i = w_begin + lane; i < w_end; i += 32) {
         const int r = r0 + i;
         int b = src[r / p.block];
         if (b < 0 || b >= nb_total(p)) {
@@ -158,7 +166,7 @@ k_attend(const AttnParams p) {
       }
     } else {
       const int32_t* src = p.idx + (size_t)(p.idx_per_group ? bkv : bh) * p.rows + r0;
-      for (int i = threadIdx.x; i < nrows; i += kAttnThreads) {
+      for (int i = w_begin + lane; i < w_end; i += 32) {
         int t = src[i];
         if (t < 0 || t >= p.T) {
           flag_status(2u);
@@ -167,7 +175,7 @@ k_attend(const AttnParams p) {
         idx_s[i] = t;
       }
     }
-    __syncthreads();
+    __syncwarp();
   }
 
   // this lane's 16 query values, pre-scaled into the log2 domain
@@ -180,12 +188,6 @@ k_attend(const AttnParams p) {
       q[2 * i + 1] = bf_hi(w[i]) * p.scale_log2;
     }
   }
-
-  // rows of this warp: [w_begin, w_end) relative to r0
-  const int rpw = ((nrows + kAttnWarps - 1) / kAttnWarps + 3) & ~3;
-  const int w_begin = min(warp * rpw, nrows);
-  const int w_end = min(w_begin + rpw, nrows);
-  const int nsteps = (w_end - w_begin + 3) >> 2;
 
   const size_t kv_base = (size_t)bkv * p.T_cap * kHeadDim;
   const uint16_t* Kh = p.K + kv_base;
