@@ -120,6 +120,7 @@ enum {
   M_NCAND = 6,                           // this CTA's candidate count
   M_LIST = 7,                            // list select: compaction counter (zero between uses)
   M_THR = 14, M_NEED = 15,               // list select: result key, its rank among equal keys
+  M_HI = 16, M_LO = 17,                  // a cluster's bracket, written by CTAs 0 and 1
   M_TOT = 8,                             // cluster totals: above, equal, cand, overflow
   M_GT_BEFORE = 12, M_EQ_BEFORE = 13     // counts of the earlier CTAs of the cluster
 };
@@ -693,7 +694,42 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
   const bool wide = cs == 1;
   uint32_t* hist0 = wide ? cand_tok : hist;
   const int hbits = wide ? kWideBits : digit_bits(0);
-  sample_pass(src, bh, T, m, whole, cand_key, hist0, 32 - hbits, scores_out, c0, len, qs);
+  if (cs > 1 && !whole) {
+    // a cluster: each CTA computes the keys of its share of the sample's
+    // blocks, then copies the other shares from the other CTAs' shared memory
+    cg::cluster_group cl = cg::this_cluster();
+    const int nblk = m / 32;
+    auto share = [&](int c, int& a, int& b) {
+      a = (c * nblk / cs) * 32;
+      b = ((c + 1) * nblk / cs) * 32;
+    };
+    int j0, j1;
+    share(rank, j0, j1);
+    const int q32 = T >> 5;
+    src.stream(bh, T, j1 - j0,
+               [&](int j) {
+                 const int jj = j0 + j;
+                 return ((int)((long long)(jj >> 5) * q32 / kSampleBlocks) << 5) + (jj & 31);
+               },
+               [&](bool v, int j, uint32_t key, float) {
+                 if (v) cand_key[j0 + j] = key;
+               },
+               qs);
+    cl.sync();  // every share is written
+    for (int c = 0; c < cs; ++c) {
+      if (c == rank) continue;
+      int a, b;
+      share(c, a, b);
+      const uint4* rk = reinterpret_cast<const uint4*>(cl.map_shared_rank(cand_key, c));
+      uint4* lk = reinterpret_cast<uint4*>(cand_key);
+      for (int i = a / 4 + threadIdx.x; i < b / 4; i += kTopkThreads) lk[i] = rk[i];
+    }
+    cl.sync();  // every copy is done before any CTA reuses its keys
+    for (int j = threadIdx.x; j < m; j += kTopkThreads)
+      atomicAdd(&hist0[cand_key[j] >> (32 - hbits)], 1u);
+  } else {
+    sample_pass(src, bh, T, m, whole, cand_key, hist0, 32 - hbits, scores_out, c0, len, qs);
+  }
   __syncthreads();
 
   // ---- 2. bracket ----------------------------------------------------------------
@@ -728,12 +764,31 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
     const int bh0 = (int)misc[M_BIN], bl0 = (int)misc[M_BIN2];
     const uint32_t ah = misc[M_ABOVE], nh = misc[M_CNT], al = misc[M_ABOVE2], nl = misc[M_CNT2];
     auto no_tok = [](int) { return 0; };
-    hi = rh ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rh, hbits, bh0, ah, nh, hist,
-                                        lists, misc, gtm, eqm, c0, len, need_unused)
-            : 0xffffffffu;
-    lo = rl ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rl, hbits, bl0, al, nl, hist,
-                                        lists, misc, gtm, eqm, c0, len, need_unused)
-            : 0u;
+    if (cs > 1) {
+      // a cluster: CTA 0 selects hi and CTA 1 lo at the same time, and each
+      // writes its key into every CTA's misc[M_HI + rank]
+      cg::cluster_group cl = cg::this_cluster();
+      uint32_t key = 0u;
+      const bool mine = (rank == 0 && rh) || (rank == 1 && rl);
+      if (rank == 0 && rh)
+        key = list_select<false, false>(cand_key, no_tok, m, 32, 0u, rh, hbits, bh0, ah, nh, hist,
+                                        lists, misc, gtm, eqm, c0, len, need_unused);
+      else if (rank == 1 && rl)
+        key = list_select<false, false>(cand_key, no_tok, m, 32, 0u, rl, hbits, bl0, al, nl, hist,
+                                        lists, misc, gtm, eqm, c0, len, need_unused);
+      if (mine && threadIdx.x == 0)
+        for (int c = 0; c < cs; ++c) cl.map_shared_rank(misc, c)[M_HI + rank] = key;
+      cl.sync();
+      hi = rh ? misc[M_HI] : 0xffffffffu;
+      lo = rl ? misc[M_LO] : 0u;
+    } else {
+      hi = rh ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rh, hbits, bh0, ah, nh,
+                                          hist, lists, misc, gtm, eqm, c0, len, need_unused)
+              : 0xffffffffu;
+      lo = rl ? list_select<false, false>(cand_key, no_tok, m, 32, 0u, rl, hbits, bl0, al, nl,
+                                          hist, lists, misc, gtm, eqm, c0, len, need_unused)
+              : 0u;
+    }
   }
 
   // ---- 3/4. stream and check; exact refinement if the bracket fails -----------
