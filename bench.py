@@ -333,12 +333,14 @@ def time_device(step: Step, steps: int, warmup: int):
 
 
 def time_e2e(step: Step, steps: int, warmup: int):
-    """Same step through the public API with host buffers: H2D of the query and of
-    the new token's K/V rows (into the caches at position T-1), the step, D2H of O.
+    """Same step through the public API with host buffers: the new token's K/V rows
+    are written into the caches at position T-1 by ds_kv_append straight from
+    pinned host memory, and ds_decode_step reads the query from pinned host
+    memory and writes O into pinned host memory (all across the host link).
 
-    The copies and the step are captured in one CUDA graph with timing events at
-    its ends (a decode loop replays such a graph every token), so the time is the
-    GPU's, copies included, without host launch gaps."""
+    The calls are captured in one CUDA graph with timing events at its ends (a
+    decode loop replays such a graph every token), so the time is the GPU's,
+    transfers included, without host launch gaps."""
     import torch
 
     w = step.w
@@ -346,25 +348,20 @@ def time_e2e(step: Step, steps: int, warmup: int):
     q_h = step.Q.cpu().pin_memory()
     kv_h = [c[:, :, w.T - 1, :].contiguous().cpu().pin_memory() for c in (step.K, step.V)]
     o_h = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
-    cudart = ctypes.CDLL("libcudart.so.12")
-    cudart.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
-                                         ctypes.c_size_t, ctypes.c_size_t, ctypes.c_size_t,
-                                         ctypes.c_int, ctypes.c_void_p]
-    row = w.d * 2
     e0 = torch.cuda.Event(enable_timing=True, external=True)
     e1 = torch.cuda.Event(enable_timing=True, external=True)
+    ds = step.ds
 
     def copies_and_step():
-        stream = torch.cuda.current_stream()
-        step.Q.copy_(q_h, non_blocking=True)
-        for src, cache in zip(kv_h, (step.K, step.V)):
-            rc = cudart.cudaMemcpy2DAsync(cache.data_ptr() + (w.T - 1) * row, w.T * row,
-                                          src.data_ptr(), row, row, w.B * w.Hkv, 1,
-                                          stream.cuda_stream)
-            assert rc == 0, rc
-        for s in step.stages():
-            s()
-        o_h.copy_(step.O, non_blocking=True)
+        ds.kv_append(kv_h[0], kv_h[1], step.K, step.V, w.T - 1)
+        if step.mode == "step":
+            ds.decode_step(q_h, step.K, step.V, step.C, step.label, step.idx, o_h, w.T,
+                           w.scale, append=True, ws=step.ws)
+        else:  # the separate calls take device buffers: copy the query in, O out
+            step.Q.copy_(q_h, non_blocking=True)
+            for s in step.stages():
+                s()
+            o_h.copy_(step.O, non_blocking=True)
 
     copies_and_step()
     torch.cuda.synchronize()

@@ -40,6 +40,9 @@
  *     ds_label_append (Double Sparsity page, Abstract and Experimental
  *     highlights: combined with offloading the KV cache to host memory).
  *     Other host memory is refused with DS_ERR_INVALID_ARG before launch.
+ *     ds_decode_step also takes Q, O and lse in such host memory: a decode
+ *     loop then hands the step its query and reads its result with no copy
+ *     of their own (the kernel reads Q and writes O over the host link).
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns DS_ERR_INVALID_ARG (or DS_ERR_UNSUPPORTED for a valid
  *     but unimplemented shape) and launches nothing.
@@ -93,9 +96,22 @@ enum {
 /* Device status bits (ds_device_status). */
 enum {
   DS_DEV_BAD_CHANNEL = 1u, /* a channel id in C was outside [0, d); masked  */
-  DS_DEV_BAD_INDEX = 2u,   /* a token index was outside [0, T); clamped     */
-  DS_DEV_TIMEOUT = 4u      /* a bounded wait on an asynchronous copy gave up  */
+  DS_DEV_BAD_INDEX = 2u    /* a token index was outside [0, T); clamped     */
 };
+
+/*
+ * ds_kv_append -- write one decode step's new K and V rows into the caches.
+ *
+ * K[b,g,t,:] = K_new[b,g,:] and V[b,g,t,:] = V_new[b,g,:] for every b, g.
+ * K_new, V_new: [B, Hkv, d] bf16, device memory or page-locked host memory
+ * mapped into the device (read directly; no separate host-to-device copy).
+ * K, V: the caches, as for ds_sparse_decode (device or mapped host memory).
+ * Requires 0 <= t < T_cap.  Bit-exact copy; one launch.  A decode step then
+ * appends the label row of token t (ds_label_append, or ds_decode_step with
+ * append) and attends with T = t + 1.
+ */
+ds_status ds_kv_append(const void* K_new, const void* V_new, void* K, void* V, ds_dims dims,
+                       int32_t t, ds_stream_t stream);
 
 /*
  * ds_label_append -- build or extend the label cache.

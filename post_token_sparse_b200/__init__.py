@@ -77,6 +77,7 @@ def _load():
         "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
         "ds_hier_score_topk": [vp, vp, vp, vp, Dims, i32, i32, vp],
+        "ds_kv_append": [vp, vp, vp, vp, Dims, i32, vp],
         "ds_block_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, i32, ctypes.c_float,
                                    vp, ctypes.c_size_t, vp],
         "ds_group_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, vp,
@@ -111,15 +112,17 @@ def lib():
 # ---------------------------------------------------------------------------
 # marshalling helpers
 
-def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor", host_ok=False):
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    # K and V may also be pinned host tensors (KV offload; see include/ds.h)
-    if not t.is_cuda and not (name in ("K", "V") and t.is_pinned()):
+    # K and V (and a decode step's Q, O, lse) may also be pinned host tensors
+    # (see include/ds.h)
+    host_ok = host_ok or name in ("K", "V")
+    if not t.is_cuda and not (host_ok and t.is_pinned()):
         raise TypeError(f"{name} must be a CUDA tensor" +
-                        (" or a pinned host tensor" if name in ("K", "V") else ""))
+                        (" or a pinned host tensor" if host_ok else ""))
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -158,6 +161,17 @@ def workspace(op: int, dims: Dims, T: int, k: int, device) -> torch.Tensor | Non
 
 # ---------------------------------------------------------------------------
 # the calls
+
+def kv_append(K_new, V_new, K, V, t: int, stream_device=None):
+    """K[:, :, t] = K_new and V[:, :, t] = V_new (K_new/V_new [B,Hkv,d] may be pinned host)."""
+    B, Hkv, T_cap, d = K.shape
+    dims = Dims(B, Hkv, Hkv, d, T_cap, 1)
+    dev = stream_device if stream_device is not None else (
+        K.device if K.is_cuda else torch.device("cuda", torch.cuda.current_device()))
+    _check(_lib.ds_kv_append(_ptr(K_new, torch.bfloat16, "K"), _ptr(V_new, torch.bfloat16, "V"),
+                             _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"), dims, t,
+                             _stream(dev)), "ds_kv_append")
+
 
 def label_append(K, C, label, t0: int, n: int):
     B, Hkv, T_cap, d = K.shape
@@ -218,15 +232,15 @@ def decode_step(Q, K, V, C, label, idx, O, T: int, scale: float, append: bool = 
     dims = dims_of(Q, K, C.shape[1])
     k = idx.shape[-1]
     if ws is None:
-        ws = workspace(OP_DECODE_STEP, dims, T, k, Q.device)
+        ws = workspace(OP_DECODE_STEP, dims, T, k, label.device)
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
-    _check(_lib.ds_decode_step(_ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"),
+    _check(_lib.ds_decode_step(_ptr(Q, torch.bfloat16, "Q", True), _ptr(K, torch.bfloat16, "K"),
                                _ptr(V, torch.bfloat16, "V"), _ptr(C, torch.int32, "C"),
                                _ptr(label, torch.bfloat16, "label"),
-                               _ptr(idx, torch.int32, "idx"), _ptr(O, torch.float32, "O"),
-                               _ptr(lse, torch.float32, "lse"), dims, T, k, scale,
+                               _ptr(idx, torch.int32, "idx"), _ptr(O, torch.float32, "O", True),
+                               _ptr(lse, torch.float32, "lse", True), dims, T, k, scale,
                                int(bool(append)), _ptr(ws, None, "ws"), nbytes,
-                               _stream(Q.device)), "ds_decode_step")
+                               _stream(label.device)), "ds_decode_step")
 
 
 def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):

@@ -51,6 +51,13 @@ ds_status check_kv(const void* K, const void* V) {
   return s != DS_OK || V == nullptr ? s : check_kv_ptr(V);
 }
 
+// ds_decode_step also takes its query and its outputs in mapped host memory:
+// the step's input and result then cross the host link inside the kernel.
+ds_status check_io(const void* Q, const void* O, const void* lse) {
+  ds_status s = check_kv(Q, O);
+  return s != DS_OK || lse == nullptr ? s : check_kv_ptr(lse);
+}
+
 ds_status cuda_fail(cudaError_t e) {
   std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e),
                 cudaGetErrorString(e));
@@ -639,6 +646,8 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
   }
   s = check_kv(K, V);
   if (s != DS_OK) return s;
+  s = check_io(Q, O, lse);
+  if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   if (fused) {
@@ -875,4 +884,22 @@ extern "C" ds_status ds_hier_score_topk(const void* Q, const int32_t* C, const v
     case 64: return launch_hier<64>(Qb, C, Lb, idx, dims, T, k, stream);
     default: return launch_hier<128>(Qb, C, Lb, idx, dims, T, k, stream);
   }
+}
+
+extern "C" ds_status ds_kv_append(const void* K_new, const void* V_new, void* K, void* V,
+                                  ds_dims dims, int32_t t, ds_stream_t stream) {
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!K_new || !V_new || !K || !V || !aligned16(K_new) || !aligned16(V_new) || !aligned16(K) ||
+      !aligned16(V))
+    return DS_ERR_INVALID_ARG;
+  if (t < 0 || t >= dims.T_cap) return DS_ERR_INVALID_ARG;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
+  s = check_kv(K_new, V_new);
+  if (s != DS_OK) return s;
+  k_kv_append<<<dims.B * dims.Hkv, 32, 0, stream>>>(
+      static_cast<const uint16_t*>(K_new), static_cast<const uint16_t*>(V_new),
+      static_cast<uint16_t*>(K), static_cast<uint16_t*>(V), dims.T_cap, t);
+  return launched();
 }

@@ -54,3 +54,22 @@ k_label_append(const uint16_t* __restrict__ K, const int32_t* __restrict__ C,
 }
 
 }  // namespace ds
+
+namespace ds {
+
+// KV-cache append of one decode step: K[b,g,t,:] = K_new[b,g,:] and the same
+// for V.  The new rows may be read from page-locked host memory mapped into
+// the device (the step's inputs arriving from the host need no copy of their
+// own).  grid (B*Hkv), 32 threads: lanes 0-15 copy the K row, 16-31 the V row,
+// 16 bytes each.
+__global__ void __launch_bounds__(32)
+k_kv_append(const uint16_t* __restrict__ K_new, const uint16_t* __restrict__ V_new,
+            uint16_t* __restrict__ K, uint16_t* __restrict__ V, int T_cap, int t) {
+  const int bg = blockIdx.x, lane = threadIdx.x;
+  const bool isv = lane >= 16;
+  const uint4* src = reinterpret_cast<const uint4*>((isv ? V_new : K_new) + (size_t)bg * kHeadDim);
+  uint4* dst = reinterpret_cast<uint4*>((isv ? V : K) + ((size_t)bg * T_cap + t) * kHeadDim);
+  dst[lane & 15] = src[lane & 15];
+}
+
+}  // namespace ds

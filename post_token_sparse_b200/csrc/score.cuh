@@ -53,19 +53,6 @@ __device__ __forceinline__ float chunk_dot(const uint4& x, const float* q) {
   return a;
 }
 
-// One thread, whole row in registers (the same tree as the lane butterfly).
-template <int R>
-__device__ __forceinline__ float row_score(const uint4 (&v)[R / 8], const float* qs) {
-  float part[R / 8];
-#pragma unroll
-  for (int c = 0; c < R / 8; ++c) part[c] = chunk_dot(v[c], qs + 8 * c);
-#pragma unroll
-  for (int st = 1; st < R / 8; st <<= 1)
-#pragma unroll
-    for (int c = 0; c < R / 8; c += 2 * st) part[c] = part[c] + part[c + st];
-  return part[0];
-}
-
 // r/8 consecutive lanes hold the chunks of one row: butterfly sum of the chunk dots.
 template <int R>
 __device__ __forceinline__ float lane_group_score(const uint4& x, const float* qs, int chunk) {

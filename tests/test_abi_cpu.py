@@ -211,6 +211,18 @@ def test_block_calls_validation():
                                       NUL) == ds.DS_ERR_WORKSPACE
 
 
+def test_kv_append_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
+    mis = ctypes.c_void_p(FAKE + 4)
+    assert lib.ds_kv_append(P, P, P, P, d, -1, NUL) == bad
+    assert lib.ds_kv_append(P, P, P, P, d, 1000, NUL) == bad
+    assert lib.ds_kv_append(NUL, P, P, P, d, 0, NUL) == bad
+    assert lib.ds_kv_append(P, P, mis, P, d, 0, NUL) == bad
+    assert lib.ds_kv_append(P, P, P, P, _dims(d=64, r=8), 0, NUL) == ds.DS_ERR_UNSUPPORTED
+
+
 def test_hier_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG

@@ -60,3 +60,46 @@ def test_offloaded_kv_matches_device_kv(shape):
     assert np.abs(host[2].cpu().numpy() - ref_O).max() <= 1e-2
     assert ds.device_status() == 0
     inp.free()
+
+
+def test_kv_append_from_device_and_pinned_host():
+    B, Hkv, T_cap, d = 2, 3, 50, 128
+    K = torch.randn(B, Hkv, T_cap, d, device="cuda").to(torch.bfloat16)
+    V = torch.randn(B, Hkv, T_cap, d, device="cuda").to(torch.bfloat16)
+    K0, V0 = K.clone(), V.clone()
+    kn = torch.randn(B, Hkv, d).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, d).to(torch.bfloat16)
+    ds.kv_append(kn.cuda(), vn.cuda(), K, V, 7)             # device source
+    ds.kv_append(kn.pin_memory(), vn.pin_memory(), K, V, 49)  # pinned host source
+    torch.cuda.synchronize()
+    for t in (7, 49):
+        assert torch.equal(K[:, :, t].cpu(), kn) and torch.equal(V[:, :, t].cpu(), vn)
+    keep = [t for t in range(T_cap) if t not in (7, 49)]
+    assert torch.equal(K[:, :, keep], K0[:, :, keep]) and torch.equal(V[:, :, keep], V0[:, :, keep])
+
+
+@pytest.mark.parametrize("shape", [(8, 32, 32, 4096, 16, 256), (1, 4, 2, 40000, 8, 10000)],
+                         ids=["one-launch", "separate-kernels"])
+def test_decode_step_with_query_and_output_in_host_memory(shape):
+    B, Hq, Hkv, T, r, k = shape
+    w = dsgen.Workload("host-io", B=B, Hq=Hq, Hkv=Hkv, T=T, r=r, k=k, n_out=min(16, r),
+                       seed=0x10 + T)
+    inp = gu.Inputs(w)
+    label = torch.empty((B, Hq, T, r), dtype=torch.bfloat16, device="cuda")
+    ds.label_append(inp.dK, inp.dC, label, 0, T - 1)
+    BH = B * Hq
+
+    def run(Q, O, lse):
+        lab = label.clone()
+        idx = torch.empty((BH, k), dtype=torch.int32, device="cuda")
+        ds.decode_step(Q, inp.dK, inp.dV, inp.dC, lab, idx, O, T, w.scale, append=True, lse=lse)
+        torch.cuda.synchronize()
+        return idx, O.cpu(), lse.cpu()
+
+    dev = run(inp.dQ, torch.empty((B, Hq, w.d), device="cuda"), torch.empty((B, Hq), device="cuda"))
+    host = run(inp.dQ.cpu().pin_memory(), torch.empty((B, Hq, w.d)).pin_memory(),
+               torch.empty((B, Hq)).pin_memory())
+    for a, b in zip(dev, host):
+        assert torch.equal(a.cpu(), b.cpu())
+    assert ds.device_status() == 0
+    inp.free()
