@@ -30,6 +30,13 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
+// Asks L2 to fetch the 128-byte line holding p from device memory.  A hint:
+// nothing waits for it, and later loads of the line find it in L2 (or meet it
+// in flight).
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Asynchronous 16-byte global->shared copy, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));

@@ -34,21 +34,28 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // device's address space (the KV cache offloaded to the host; kernels then
 // read the rows they need over the host link).  Any other host memory is
 // refused before a launch could touch it.  When the runtime cannot be asked
-// (no device), the launch itself reports the error.
-ds_status check_kv_ptr(const void* p) {
+// (no device), the launch itself reports the error.  *device (optional): p is
+// plain device memory.
+ds_status check_kv_ptr(const void* p, bool* device = nullptr) {
+  if (device) *device = false;
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
     cudaGetLastError();
     return DS_OK;
   }
+  if (device) *device = a.type == cudaMemoryTypeDevice;
   if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return DS_OK;
   if (a.type == cudaMemoryTypeHost && a.devicePointer == p) return DS_OK;
   return DS_ERR_INVALID_ARG;
 }
 
-ds_status check_kv(const void* K, const void* V) {
-  ds_status s = check_kv_ptr(K);
-  return s != DS_OK || V == nullptr ? s : check_kv_ptr(V);
+// *device (optional): K and V are both plain device memory.
+ds_status check_kv(const void* K, const void* V, bool* device = nullptr) {
+  bool dk = false, dv = true;
+  ds_status s = check_kv_ptr(K, &dk);
+  if (s == DS_OK && V != nullptr) s = check_kv_ptr(V, &dv);
+  if (device) *device = dk && dv;
+  return s;
 }
 
 // ds_decode_step also takes its query and its outputs in mapped host memory:
@@ -644,7 +651,8 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
                      dims.r == 128;
     if (!vec) return DS_ERR_UNSUPPORTED;  // the fused score+select needs a vector path
   }
-  s = check_kv(K, V);
+  bool kv_device = false;
+  s = check_kv(K, V, &kv_device);
   if (s != DS_OK) return s;
   s = check_io(Q, O, lse);
   if (s != DS_OK) return s;
@@ -666,6 +674,7 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
     sp.T = T;
     sp.k = k;
     sp.append = append ? 1 : 0;
+    sp.prefetch = kv_device ? 1 : 0;
     sp.scale_log2 = scale * 1.4426950408889634f;
     const int BH = dims.B * dims.Hq;
     switch (dims.r) {

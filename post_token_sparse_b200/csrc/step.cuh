@@ -37,7 +37,27 @@ struct StepParams {
   float* O;
   float* lse;    // optional
   int Hq, Hkv, T_cap, T, k, append;
+  int prefetch;  // K and V are in device memory: rows sure to be kept are
+                 // prefetched into L2 while the selection finishes
   float scale_log2;
+};
+
+// The K and V rows of the tokens the selection has already settled on are
+// asked into L2 (two 128-byte lines per 256-byte row), so that the attention
+// phase finds most of its rows there instead of waiting on HBM after the
+// selection; the HBM reads overlap the selection's on-chip work.
+struct PrefetchSureRows {
+  const uint16_t* K;  // row 0 of this KV head; null: no prefetch
+  const uint16_t* V;
+  __device__ __forceinline__ void operator()(int t) const {
+    if (K == nullptr) return;
+    const char* k = reinterpret_cast<const char*>(K + (size_t)t * kHeadDim);
+    const char* v = reinterpret_cast<const char*>(V + (size_t)t * kHeadDim);
+    prefetch_l2_line(k);
+    prefetch_l2_line(k + 128);
+    prefetch_l2_line(v);
+    prefetch_l2_line(v + 128);
+  }
 };
 
 // Shared memory of the step kernel in 32-bit words: the selection's layout,
@@ -209,8 +229,10 @@ k_step(const StepParams p, int chunk) {
     src.over_t = p.T - 1;
     src.over_row = reinterpret_cast<const uint4*>(over16);
   }
+  const size_t kv = (size_t)bkv * p.T_cap * kHeadDim;
+  const PrefetchSureRows pf{p.prefetch ? p.K + kv : nullptr, p.V + kv};
   topk_body(src, sm, 1, 0, bh, p.T, p.k, chunk, p.idx ? p.idx + (size_t)bh * p.k : nullptr,
-            idx_s, true);
+            idx_s, true, pf);
   __syncthreads();
 
   // 3. attention over the kept rows (the selection's shared memory is free now)

@@ -427,6 +427,13 @@ __device__ __forceinline__ void rank_in_list(const uint32_t* sk, int ns, uint32_
   __syncthreads();
 }
 
+// Called once for every token that the selection of a whole-head sample has
+// settled on before the exact threshold is known: its key lies in a higher bin
+// of the first digit than the k-th key's (token t: item t of the key array).
+struct NoSureHook {
+  __device__ __forceinline__ void operator()(int) const {}
+};
+
 // List select: the key of rank r (1 = largest) among the live items of a key
 // array in shared memory.  Source item i < n has key key0[i] and token tok0(i);
 // the live items are those that carry the prefix pf above bit `top` (top = 32:
@@ -438,14 +445,15 @@ __device__ __forceinline__ void rank_in_list(const uint32_t* sk, int ns, uint32_
 // of 32.  n <= 4 * kSelectIters * kTopkThreads, key0 16-byte aligned, and key0
 // readable up to n rounded up to 4.  need: the result's rank among the
 // keys equal to it.  misc[M_LIST] is zero on entry and on exit.  Block-uniform.
-template <bool kCls, bool kSeqTok, class TokFn>
+template <bool kCls, bool kSeqTok, class TokFn, class SureHook = NoSureHook>
 __device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0, int n, int top,
                                                 uint32_t pf, uint32_t r, int first_bits,
                                                 int first_bin, uint32_t first_above,
                                                 uint32_t first_cnt,
                                                 uint32_t* hist, uint32_t* lists, uint32_t* misc,
                                                 uint32_t* gtm, uint32_t* eqm, int c0, int len,
-                                                uint32_t& need) {
+                                                uint32_t& need,
+                                                const SureHook& on_sure = SureHook()) {
   const int lane = threadIdx.x & 31;
   const uint32_t* sk = key0;
   const uint32_t* st = nullptr;  // tokens of the current list (null: the source array)
@@ -511,6 +519,9 @@ __device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0
             wm |= __shfl_xor_sync(0xffffffffu, wm, 4);
             const int j = i0 - 4 * (lane & 7) - c0;
             if ((lane & 7) == 0 && wm && j >= 0 && j < len) gtm[j >> 5] |= wm;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if ((up >> u) & 1u) on_sure(i0 + u);
           } else {
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -579,9 +590,9 @@ __device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0
 
 // The streaming passes of the kernel below.
 
-// Sample pass: keys of the m sampled tokens into keys[], the histogram of
-// their top 32 - hshift bits into hist; scores of this CTA's tokens when the
-// whole head is the sample.
+// Sample pass (block-uniform): keys of the m sampled tokens into keys[], the
+// histogram of their top 32 - hshift bits into hist; scores of this CTA's
+// tokens when the whole head is the sample.
 template <class Source>
 __device__ __forceinline__ void sample_pass(const Source& src, int bh, int T, int m, bool whole,
                                          uint32_t* keys, uint32_t* hist, int hshift,
@@ -594,11 +605,14 @@ __device__ __forceinline__ void sample_pass(const Source& src, int bh, int T, in
              [&](bool v, int j, uint32_t key, float s) {
                if (v) {
                  keys[j] = key;
-                 atomicAdd(&hist[key >> hshift], 1u);
                  if (whole && scores_out && j >= c0 && j < c0 + len) scores_out[j] = s;
                }
              },
              qs);
+  // the histogram from shared memory once every key is in: no shared-memory
+  // atomics between the loads of the stream
+  __syncthreads();
+  for (int j = threadIdx.x; j < m; j += kTopkThreads) atomicAdd(&hist[keys[j] >> hshift], 1u);
 }
 
 // Main pass over this CTA's tokens against the bracket [lo, hi].
@@ -654,10 +668,12 @@ __device__ __forceinline__ void digit_hist_pass(const Source& src, int bh, int T
 // selected indices, ascending, go to dst_g (global, k entries) and/or dst_s
 // (shared memory, k entries); either may be null.  qs_ready: the caller has
 // already written the source's query values (TopkLayout::small + 64 onwards).
-template <class Source>
+// on_sure: see NoSureHook (called only when T <= kSample).
+template <class Source, class SureHook = NoSureHook>
 __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int cs, int rank,
                                           int bh, int T, int k, int chunk, int32_t* dst_g,
-                                          int32_t* dst_s, bool qs_ready = false) {
+                                          int32_t* dst_s, bool qs_ready = false,
+                                          const SureHook& on_sure = SureHook()) {
   const TopkLayout L(chunk, cs);
   uint32_t* hist = sm;
   uint32_t* misc = sm + L.small;
@@ -748,7 +764,7 @@ __device__ __forceinline__ void topk_body(const Source& src, uint32_t* sm, int c
     const uint32_t a0 = misc[M_ABOVE], n0 = misc[M_CNT];
     const uint32_t thr = list_select<true, true>(
         cand_key, [](int i) { return i; }, T, 32, 0u, (uint32_t)k, hbits, b0, a0, n0, hist,
-        lists, misc, gtm, eqm, c0, len, need_unused);
+        lists, misc, gtm, eqm, c0, len, need_unused, on_sure);
     lo = hi = thr;
   } else {
     const float e = (float)k * (float)m / (float)T;
