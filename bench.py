@@ -333,10 +333,11 @@ def time_device(step: Step, steps: int, warmup: int):
 
 
 def time_e2e(step: Step, steps: int, warmup: int):
-    """Same step through the public API with host buffers: the new token's K/V rows
-    are written into the caches at position T-1 by ds_kv_append straight from
-    pinned host memory, and ds_decode_step reads the query from pinned host
-    memory and writes O into pinned host memory (all across the host link).
+    """Same step through the public API with host buffers: ds_decode_step_kv takes
+    the new token's K/V rows and the query from pinned host memory, stores the
+    rows into the caches at position T-1, and writes O into pinned host memory
+    (all across the host link, inside the one step launch).  The separate-call
+    path stores the rows with ds_kv_append and copies the query in and O out.
 
     The calls are captured in one CUDA graph with timing events at its ends (a
     decode loop replays such a graph every token), so the time is the GPU's,
@@ -353,11 +354,11 @@ def time_e2e(step: Step, steps: int, warmup: int):
     ds = step.ds
 
     def copies_and_step():
-        ds.kv_append(kv_h[0], kv_h[1], step.K, step.V, w.T - 1)
         if step.mode == "step":
-            ds.decode_step(q_h, step.K, step.V, step.C, step.label, step.idx, o_h, w.T,
-                           w.scale, append=True, ws=step.ws)
+            ds.decode_step_kv(q_h, kv_h[0], kv_h[1], step.K, step.V, step.C, step.label,
+                              step.idx, o_h, w.T, w.scale, ws=step.ws)
         else:  # the separate calls take device buffers: copy the query in, O out
+            ds.kv_append(kv_h[0], kv_h[1], step.K, step.V, w.T - 1)
             step.Q.copy_(q_h, non_blocking=True)
             for s in step.stages():
                 s()

@@ -222,6 +222,32 @@ ds_status ds_decode_step(const void* Q, const void* K, const void* V, const int3
                          size_t ws_bytes, ds_stream_t stream);
 
 /*
+ * ds_decode_step_kv -- ds_decode_step for a decoder that hands over the newest
+ * token's K and V rows with the step.
+ *
+ * Exactly ds_kv_append(K_new, V_new, K, V, dims, T-1) followed by
+ * ds_decode_step(Q, K, V, C, label, idx, O, lse, dims, T, k, scale, 1, ...):
+ * the new rows are stored at t = T-1, the label row of t = T-1 is appended,
+ * then top-k selection and sparse attention over the T tokens.  Where
+ * ds_decode_step runs as one launch, so does this call: the new rows are
+ * stored by the step kernel itself, which also reads token T-1's rows from
+ * K_new / V_new.  The online inference phase of Double Sparsity (page, Method
+ * details: Technical framework) runs once per generated token; storing that
+ * token's K and V first is ordinary decoder bookkeeping, which the pages do
+ * not describe (the plainest reading: the new token is attended to).
+ *
+ * K_new, V_new: [B, Hkv, d] bf16, device memory or page-locked host memory
+ * mapped into the device; they must not overlap K, V or label.  K, V: the
+ * caches, written in row T-1 only.  Requires 1 <= T <= T_cap.  Q, O and lse
+ * may be mapped host memory as for ds_decode_step; other arguments, results,
+ * errors and the workspace (DS_OP_DECODE_STEP) as for ds_decode_step.
+ */
+ds_status ds_decode_step_kv(const void* Q, const void* K_new, const void* V_new, void* K,
+                            void* V, const int32_t* C, void* label, int32_t* idx, float* O,
+                            float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
+                            void* ws, size_t ws_bytes, ds_stream_t stream);
+
+/*
  * ds_decode -- dense decode attention over all T cached tokens: the operation
  * token sparsity accelerates (Double Sparsity page, Experimental highlights:
  * attention-operation speed-up).  Same as ds_sparse_decode with

@@ -73,6 +73,8 @@ def _load():
         "ds_device_status": [u32p, i32, vp],
         "ds_decode_step": [vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, i32,
                            vp, ctypes.c_size_t, vp],
+        "ds_decode_step_kv": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32,
+                              ctypes.c_float, vp, ctypes.c_size_t, vp],
         "ds_calibrate": [vp, i32, vp, Dims, i32, vp, vp, vp, ctypes.c_size_t, vp],
         "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
@@ -241,6 +243,27 @@ def decode_step(Q, K, V, C, label, idx, O, T: int, scale: float, append: bool = 
                                _ptr(lse, torch.float32, "lse", True), dims, T, k, scale,
                                int(bool(append)), _ptr(ws, None, "ws"), nbytes,
                                _stream(label.device)), "ds_decode_step")
+
+
+def decode_step_kv(Q, K_new, V_new, K, V, C, label, idx, O, T: int, scale: float, lse=None,
+                   ws=None):
+    """decode_step with the newest token's K/V rows handed over: K[:, :, T-1] = K_new,
+    V[:, :, T-1] = V_new, then the step with append (K_new/V_new [B,Hkv,d] may be pinned host)."""
+    dims = dims_of(Q, K, C.shape[1])
+    k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_DECODE_STEP, dims, T, k, label.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_decode_step_kv(_ptr(Q, torch.bfloat16, "Q", True),
+                                  _ptr(K_new, torch.bfloat16, "K_new", True),
+                                  _ptr(V_new, torch.bfloat16, "V_new", True),
+                                  _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
+                                  _ptr(C, torch.int32, "C"), _ptr(label, torch.bfloat16, "label"),
+                                  _ptr(idx, torch.int32, "idx"),
+                                  _ptr(O, torch.float32, "O", True),
+                                  _ptr(lse, torch.float32, "lse", True), dims, T, k, scale,
+                                  _ptr(ws, None, "ws"), nbytes, _stream(label.device)),
+           "ds_decode_step_kv")
 
 
 def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):

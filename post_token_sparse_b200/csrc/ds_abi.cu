@@ -626,11 +626,13 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
 }
 
-extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
-                                    void* label, int32_t* idx, float* O, float* lse,
-                                    ds_dims dims, int32_t T, int32_t k, float scale,
-                                    int32_t append, void* ws, size_t ws_bytes,
-                                    ds_stream_t stream) {
+namespace {
+
+// ds_decode_step, and ds_decode_step_kv when K_new is given (then append is 1).
+ds_status decode_step(const void* Q, const void* K_new, const void* V_new, const void* K,
+                      const void* V, const int32_t* C, void* label, int32_t* idx, float* O,
+                      float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
+                      int32_t append, void* ws, size_t ws_bytes, ds_stream_t stream) {
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !C || !label || !idx || !O || !aligned16(Q) || !aligned16(K) ||
@@ -638,6 +640,11 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
       (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (K_new) {
+    if (!V_new || !aligned16(K_new) || !aligned16(V_new)) return DS_ERR_INVALID_ARG;
+    s = check_kv(K_new, V_new);
+    if (s != DS_OK) return s;
+  }
   if (T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
   int chunk = 0;
   size_t smem = 0;
@@ -663,6 +670,8 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
     sp.Q = static_cast<const uint16_t*>(Q);
     sp.K = static_cast<const uint16_t*>(K);
     sp.V = static_cast<const uint16_t*>(V);
+    sp.K_new = static_cast<const uint16_t*>(K_new);
+    sp.V_new = static_cast<const uint16_t*>(V_new);
     sp.C = C;
     sp.label = static_cast<uint16_t*>(label);
     sp.idx = idx;
@@ -685,7 +694,12 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
       default: return launch_step<128>(sp, BH, chunk, smem, stream);
     }
   }
-  // the same step as three calls
+  // the same step as separate calls
+  if (K_new) {
+    s = ds_kv_append(K_new, V_new, const_cast<void*>(K), const_cast<void*>(V), dims, T - 1,
+                     stream);
+    if (s != DS_OK) return s;
+  }
   if (append) {
     s = ds_label_append(K, C, label, dims, T - 1, 1, stream);
     if (s != DS_OK) return s;
@@ -695,6 +709,27 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
   s = ds_score_topk(Q, C, label, scores, idx, dims, T, k, stream);
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
+}
+
+}  // namespace
+
+extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
+                                    void* label, int32_t* idx, float* O, float* lse,
+                                    ds_dims dims, int32_t T, int32_t k, float scale,
+                                    int32_t append, void* ws, size_t ws_bytes,
+                                    ds_stream_t stream) {
+  return decode_step(Q, nullptr, nullptr, K, V, C, label, idx, O, lse, dims, T, k, scale, append,
+                     ws, ws_bytes, stream);
+}
+
+extern "C" ds_status ds_decode_step_kv(const void* Q, const void* K_new, const void* V_new,
+                                       void* K, void* V, const int32_t* C, void* label,
+                                       int32_t* idx, float* O, float* lse, ds_dims dims,
+                                       int32_t T, int32_t k, float scale, void* ws,
+                                       size_t ws_bytes, ds_stream_t stream) {
+  if (!K_new || !V_new) return DS_ERR_INVALID_ARG;
+  return decode_step(Q, K_new, V_new, K, V, C, label, idx, O, lse, dims, T, k, scale, 1, ws,
+                     ws_bytes, stream);
 }
 
 extern "C" ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_dims dims,

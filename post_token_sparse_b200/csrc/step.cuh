@@ -10,7 +10,10 @@
 //               gathered into shared memory and written to the label cache;
 //               the selection reads that row from shared memory, so the kernel
 //               never reads back through the non-coherent load path a row it
-//               wrote itself
+//               wrote itself.  When the caller hands over the newest token's K
+//               and V rows (K_new, V_new), they are also stored into the K and V
+//               caches here, and the label channels and token T-1's attention
+//               rows are read from K_new / V_new
 //   2. select   the top-k body of topk.cuh; the k indices land in shared memory
 //               (and in idx when requested)
 //   3. attend   8 warps each take a contiguous run of the kept rows through a
@@ -24,6 +27,7 @@
 namespace ds {
 
 constexpr int kStepWarps = kTopkThreads / 32;  // 8
+static_assert(kTopkThreads >= kHeadDim + 32, "threads d..d+31 store the new K and V rows");
 constexpr int kStepStages = 3;
 constexpr int kStepMaxK = 8192;
 
@@ -31,6 +35,8 @@ struct StepParams {
   const uint16_t* Q;
   const uint16_t* K;
   const uint16_t* V;
+  const uint16_t* K_new;  // optional: the newest token's K and V rows [B*Hkv, d],
+  const uint16_t* V_new;  // stored into the caches at T-1 by this kernel
   const int32_t* C;
   uint16_t* label;
   int32_t* idx;  // optional copy of the selected indices [BH, k]
@@ -106,13 +112,18 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
   const uint16_t* Vh = p.V + kv_base;
   uint4* my_ring = ring + warp * kStepStages * kAttnStageU4;
 
+  // with K_new, token T-1's rows are read from there: another CTA of the KV
+  // group may not have stored them into the caches yet
+  const uint16_t* Knew = p.K_new ? p.K_new + (size_t)bkv * kHeadDim : nullptr;
+  const uint16_t* Vnew = p.K_new ? p.V_new + (size_t)bkv * kHeadDim : nullptr;
   auto issue = [&](int step) {
     const int lr = w_begin + step * 4 + g;
     if (lr < w_end) {
       int t = idx_s[lr];
       t = min(max(t, 0), p.T - 1);
-      const uint4* krow = reinterpret_cast<const uint4*>(Kh + (size_t)t * kHeadDim);
-      const uint4* vrow = reinterpret_cast<const uint4*>(Vh + (size_t)t * kHeadDim);
+      const bool nw = Knew != nullptr && t == p.T - 1;
+      const uint4* krow = reinterpret_cast<const uint4*>(nw ? Knew : Kh + (size_t)t * kHeadDim);
+      const uint4* vrow = reinterpret_cast<const uint4*>(nw ? Vnew : Vh + (size_t)t * kHeadDim);
       uint4* st = my_ring + (step % kStepStages) * kAttnStageU4 + g * 32;
       cp_async16(st + c, krow + c);
       cp_async16(st + 8 + c, krow + 8 + c);
@@ -200,11 +211,20 @@ k_step(const StepParams p, int chunk) {
   int32_t* idx_s = reinterpret_cast<int32_t*>(sm + SL.idx);
 
   // 1. the newest token's label row, and q at the label channels (one load of
-  //    each channel id serves both)
+  //    each channel id serves both); with K_new, the newest token's K and V
+  //    rows are stored into the caches by the KV group's first query head
   float* qs = reinterpret_cast<float*>(sm + TopkLayout(chunk, 1).small + 64);
   {
     const int t = p.T - 1;
-    const uint16_t* krow = p.K + ((size_t)bkv * p.T_cap + t) * kHeadDim;
+    const size_t cache_row = ((size_t)bkv * p.T_cap + t) * kHeadDim;
+    const uint16_t* krow = p.K_new ? p.K_new + (size_t)bkv * kHeadDim : p.K + cache_row;
+    if (p.K_new && h % G == 0 && threadIdx.x >= kHeadDim && threadIdx.x < kHeadDim + 32) {
+      const int i = threadIdx.x - kHeadDim;  // 16-byte chunk i % 16 of the K (i < 16) or V row
+      const uint4* src = reinterpret_cast<const uint4*>(
+          (i < 16 ? p.K_new : p.V_new) + (size_t)bkv * kHeadDim);
+      uint4* dst = reinterpret_cast<uint4*>(const_cast<uint16_t*>(i < 16 ? p.K : p.V) + cache_row);
+      dst[i & 15] = src[i & 15];
+    }
     uint16_t* lrow = p.label + ((size_t)bh * p.T_cap + t) * R;
     for (int j = threadIdx.x; j < R; j += kTopkThreads) {
       int ch = p.C[h * R + j];

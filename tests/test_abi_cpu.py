@@ -223,6 +223,30 @@ def test_kv_append_validation():
     assert lib.ds_kv_append(P, P, P, P, _dims(d=64, r=8), 0, NUL) == ds.DS_ERR_UNSUPPORTED
 
 
+def test_decode_step_kv_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
+    mis = ctypes.c_void_p(FAKE + 4)
+    #                            Q  Kn   Vn   K  V  C  lab idx O  lse  dims T  k
+    assert lib.ds_decode_step_kv(P, NUL, P, P, P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, NUL, P, P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, mis, P, P, P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, mis, P, P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, P, P, P, P, P, P, P, NUL, d, 0, 1, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, P, P, P, P, P, P, P, NUL, d, 1001, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, P, P, P, P, P, P, P, NUL, d, 10, 11, 1.0, NUL, 0,
+                                 NUL) == bad
+    assert lib.ds_decode_step_kv(P, P, P, NUL, P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0,
+                                 NUL) == bad
+
+
 def test_hier_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG

@@ -110,3 +110,67 @@ def test_decode_step_full_workload_sampled_heads(name):
         o, _, _ = oracle.attend_head(inp.Q[b, h], inp.K[b, g], inp.V[b, g], sel, w.scale)
         assert np.abs(On[b, h] - o).max() <= 1e-2
     inp.free()
+
+
+KV_CASES = [
+    # (name, B, Hq, Hkv, T, T_cap, r, k)
+    ("mha-T100-r16", 2, 3, 3, 100, 120, 16, 7),
+    ("gqa-T1000-r16", 2, 8, 2, 1000, 1003, 16, 37),    # four CTAs share each new row
+    ("mha-T1-r8", 1, 2, 2, 1, 1, 8, 1),                 # the new token is the only one
+    ("mha-T4097-r32", 1, 4, 4, 4097, 4100, 32, 300),
+    ("mha-T2500-r128-kT", 1, 2, 2, 2500, 2600, 128, 2500),  # every token kept
+    ("mha-T40000-r8-fallback", 1, 2, 2, 40000, 40000, 8, 10000),
+]
+
+
+@pytest.mark.parametrize("host", [False, True], ids=["device", "host-io"])
+@pytest.mark.parametrize("case", KV_CASES, ids=[c[0] for c in KV_CASES])
+def test_decode_step_kv_equals_kv_append_then_step(case, host):
+    """ds_decode_step_kv is ds_kv_append(T-1) followed by ds_decode_step with append:
+    the same caches, label cache and index set bit for bit, the same O to fp32
+    rounding.  The new rows differ from what the caches held at T-1, so a row not
+    stored, or token T-1 attended from the stale cache row, shows."""
+    name, B, Hq, Hkv, T, T_cap, r, k = case
+    w = dsgen.Workload(name, B=B, Hq=Hq, Hkv=Hkv, T=T_cap, r=r, k=k, n_out=min(8, r),
+                       seed=0x5EED + 7 * T)
+    inp = gu.Inputs(w, r=r)
+    g = torch.Generator(device="cpu").manual_seed(T)
+    kn = (3 * torch.randn((B, Hkv, w.d), generator=g)).to(torch.bfloat16)
+    vn = torch.randn((B, Hkv, w.d), generator=g).to(torch.bfloat16)
+    label = torch.zeros((B, Hq, T_cap, r), dtype=torch.bfloat16, device="cuda")
+    if T > 1:
+        ds.label_append(inp.dK, inp.dC, label, 0, T - 1)
+    BH = B * Hq
+    # the separate calls
+    K1, V1, L1 = inp.dK.clone(), inp.dV.clone(), label.clone()
+    ds.kv_append(kn.cuda(), vn.cuda(), K1, V1, T - 1)
+    idx1 = torch.empty((BH, k), dtype=torch.int32, device="cuda")
+    O1 = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+    ds.decode_step(inp.dQ, K1, V1, inp.dC, L1, idx1, O1, T, w.scale, append=True)
+    # the one call
+    K2, V2, L2 = inp.dK.clone(), inp.dV.clone(), label.clone()
+    idx2 = torch.full((BH, k), -1, dtype=torch.int32, device="cuda")
+    if host:
+        q, kn2, vn2 = inp.dQ.cpu().pin_memory(), kn.pin_memory(), vn.pin_memory()
+        O2 = torch.empty((B, Hq, w.d), dtype=torch.float32).pin_memory()
+        lse2 = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    else:
+        q, kn2, vn2 = inp.dQ, kn.cuda(), vn.cuda()
+        O2 = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+        lse2 = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ds.decode_step_kv(q, kn2, vn2, K2, V2, inp.dC, L2, idx2, O2, T, w.scale, lse=lse2)
+    torch.cuda.synchronize()
+    assert torch.equal(K2.view(torch.int16), K1.view(torch.int16))
+    assert torch.equal(V2.view(torch.int16), V1.view(torch.int16))
+    assert torch.equal(L2.view(torch.int16), L1.view(torch.int16))
+    assert torch.equal(idx2, idx1)
+    assert (O2.cuda() - O1).abs().max().item() <= 1e-5
+    # and the oracle on the appended caches
+    Kh = gu.host_bits(K1)
+    Vh = gu.host_bits(V1)
+    I = idx2.cpu().numpy().reshape(B, Hq, k)
+    ref_O, ref_L = oracle.attend(inp.Q, Kh, Vh, I, w.scale)
+    assert np.abs(O2.cpu().numpy() - ref_O).max() <= 1e-2
+    L = lse2.cpu().numpy()
+    assert np.all(np.abs(L - ref_L) <= 1e-3 * (1 + np.abs(ref_L)))
+    assert ds.device_status() == 0
