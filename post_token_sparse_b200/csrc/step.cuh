@@ -27,7 +27,8 @@
 namespace ds {
 
 constexpr int kStepWarps = kTopkThreads / 32;  // 8
-static_assert(kTopkThreads >= kHeadDim + 32, "threads d..d+31 store the new K and V rows");
+static_assert(kTopkThreads >= kHeadDim + 48,
+              "threads d..d+31 store the new K and V rows, d+32..d+47 load the query row");
 constexpr int kStepStages = 3;
 constexpr int kStepMaxK = 8192;
 
@@ -68,15 +69,18 @@ struct PrefetchSureRows {
 
 // Shared memory of the step kernel in 32-bit words: the selection's layout,
 // overlaid afterwards by the attention ring and warp partials; then the new
-// token's label row and the index list, which both phases use.
+// token's label row, the query row and the index list, which outlive the
+// selection.
 struct StepLayout {
-  int over, idx, words;
+  int over, q, idx, words;
   __host__ __device__ StepLayout(int chunk, int k) {
     const int sel = TopkLayout(chunk, 1).words;
     const int att = kStepWarps * kStepStages * kAttnStageU4 * 4 + kStepWarps * 132;
     int o = sel > att ? sel : att;
     o = (o + 3) & ~3;
     over = o;  // label row of the newest token (up to 128 bf16 = 64 words)
+    o += 64;
+    q = o;  // the query row (128 bf16)
     o += 64;
     idx = o;
     o += (k + 3) & ~3;
@@ -89,12 +93,11 @@ struct StepLayout {
 // bkv), by kStepWarps warps; writes O[bh] and lse[bh].
 __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv,
                                             const int32_t* idx_s, int n, uint4* ring,
-                                            float* red) {
+                                            float* red, const uint4* qrow) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 3, c = lane & 7;
   float q[16];
   {
-    const uint4* qrow = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim);
     const uint4 a = qrow[c], bq = qrow[8 + c];
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
@@ -208,6 +211,7 @@ k_step(const StepParams p, int chunk) {
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bkv = b * p.Hkv + h / G;
   uint16_t* over16 = reinterpret_cast<uint16_t*>(sm + SL.over);
+  uint4* q_s = reinterpret_cast<uint4*>(sm + SL.q);
   int32_t* idx_s = reinterpret_cast<int32_t*>(sm + SL.idx);
 
   // 1. the newest token's label row, and q at the label channels (one load of
@@ -224,6 +228,12 @@ k_step(const StepParams p, int chunk) {
           (i < 16 ? p.K_new : p.V_new) + (size_t)bkv * kHeadDim);
       uint4* dst = reinterpret_cast<uint4*>(const_cast<uint16_t*>(i < 16 ? p.K : p.V) + cache_row);
       dst[i & 15] = src[i & 15];
+    }
+    if (threadIdx.x >= kHeadDim + 32 && threadIdx.x < kHeadDim + 48) {
+      // the query row, kept for the attention phase (the selection's barriers
+      // publish it); its load overlaps the label channel loads
+      const int i = threadIdx.x - kHeadDim - 32;
+      q_s[i] = reinterpret_cast<const uint4*>(p.Q + (size_t)bh * kHeadDim)[i];
     }
     uint16_t* lrow = p.label + ((size_t)bh * p.T_cap + t) * R;
     for (int j = threadIdx.x; j < R; j += kTopkThreads) {
@@ -258,7 +268,7 @@ k_step(const StepParams p, int chunk) {
   // 3. attention over the kept rows (the selection's shared memory is free now)
   uint4* ring = reinterpret_cast<uint4*>(sm);
   float* red = reinterpret_cast<float*>(ring + kStepWarps * kStepStages * kAttnStageU4);
-  attend_rows(p, bh, bkv, idx_s, p.k, ring, red);
+  attend_rows(p, bh, bkv, idx_s, p.k, ring, red, q_s);
 }
 
 }  // namespace ds
