@@ -427,9 +427,9 @@ __device__ __forceinline__ void rank_in_list(const uint32_t* sk, int ns, uint32_
   __syncthreads();
 }
 
-// Called once for every token that the selection of a whole-head sample has
-// settled on before the exact threshold is known: its key lies in a higher bin
-// of the first digit than the k-th key's (token t: item t of the key array).
+// Called once for every token a whole-head list select settles on before the
+// exact threshold is known: at some digit its key is in a higher bin than the
+// k-th key's, all digits above being equal (token t: item t of the key array).
 struct NoSureHook {
   __device__ __forceinline__ void operator()(int) const {}
 };
@@ -443,8 +443,9 @@ struct NoSureHook {
 // their token's bit in gtm and live items equal to it in eqm (tokens of
 // [c0, c0 + len) only; bit t - c0); kSeqTok: tok0(i) == i, and c0 is a multiple
 // of 32.  n <= 4 * kSelectIters * kTopkThreads, key0 16-byte aligned, and key0
-// readable up to n rounded up to 4.  need: the result's rank among the
-// keys equal to it.  misc[M_LIST] is zero on entry and on exit.  Block-uniform.
+// readable up to n rounded up to 4.  need: the result's rank among the keys
+// equal to it.  misc[M_LIST] is zero on entry and on exit.  on_sure: see
+// NoSureHook (kCls && kSeqTok).  Block-uniform.
 template <bool kCls, bool kSeqTok, class TokFn, class SureHook = NoSureHook>
 __device__ __forceinline__ uint32_t list_select(const uint32_t* key0, TokFn tok0, int n, int top,
                                                 uint32_t pf, uint32_t r, int first_bits,
