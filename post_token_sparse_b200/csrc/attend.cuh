@@ -30,6 +30,7 @@ namespace ds {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
+static_assert(kAttnThreads == kHeadDim, "the merges give thread j output dim j");
 constexpr int kAttnStages = 4;
 constexpr int kAttnStageU4 = 4 * 32;  // 4 rows x (16 uint4 of K + 16 uint4 of V) = 2 KB
 constexpr int kPartialStride = 132;   // floats per split partial: m, l, pad, pad, o[128]
