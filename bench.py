@@ -392,9 +392,17 @@ def time_e2e(step: Step, steps: int, warmup: int):
 # the CPU oracle, timed on a bounded sample of heads
 
 def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
+    """The oracle's score + top-k + attention per head, one thread: the C++ oracle
+    (steps O1-O5), or the numpy oracle where the C++ one cannot be built."""
     import numpy as np
 
-    import oracle
+    try:
+        import oracle.cxx as oracle
+        oracle.build()
+        kind = "float64 C++ (std::sort, std::exp)"
+    except Exception:  # noqa: BLE001  (no C++ compiler: the numpy oracle, said so)
+        import oracle
+        kind = "float64 numpy"
 
     try:
         from threadpoolctl import threadpool_limits
@@ -447,7 +455,7 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
     out = {"value": per_head * done / elapsed / 1e9, "unit": "GB/s", "cores": 1,
            "kind": "oracle", "us_per_step": us_step,
            "sample": f"{done} head-steps ({passes} pass(es) over the {w.B * w.Hq} heads) of "
-                     f"{w.name}, score + top-k + attention per head in float64 numpy, one "
+                     f"{w.name}, score + top-k + attention per head in {kind}, one "
                      f"thread ({elapsed:.1f} s)"}
     if with_dense:
         out["dense_us_per_step"] = dense_el / done * w.B * w.Hq * 1e6

@@ -532,6 +532,10 @@ def pin_hier_topk(orc):
         assert len(set(got)) == k and all(0 <= t < T for t in got) and list(got) == sorted(got)
 
 
+# the pins of steps O1-O5 and the merge: also run against the C++ oracle
+CORE_PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
+             pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding]
+
 PINS = [pin_bf16, pin_label, pin_score, pin_topk, pin_attend, pin_merge, pin_dense,
         pin_full_channels_all_tokens, pin_worked_score, pin_f32_rounding,
         pin_calib_bruteforce, pin_calib_groups_and_order, pin_calib_permutation,

@@ -1,0 +1,114 @@
+"""The C++ oracle (steps O1-O5 and the merge, oracle/ds_oracle.cpp), no GPU needed.
+
+1. The same pins as the numpy oracle's steps: bf16 decoding, label gather,
+   score, top-k order and worked examples, attention against torch's
+   scaled_dot_product_attention and closed forms, merge invariance, dense,
+   r = d with k = T.
+2. Planted slips in a copy of the C++ source (compiled into a temporary
+   directory): each must make at least one of those pins fail.
+3. Agreement with the numpy oracle on seeded workloads (MHA and grouped KV
+   heads, tie-heavy scores): the two implementations share no code.
+"""
+import importlib.util
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+import dsgen
+import oracle
+import oracle.cxx as cxx
+from tests import pins
+
+
+@pytest.mark.parametrize("pin", pins.CORE_PINS, ids=lambda p: p.__name__)
+def test_cxx_pin(pin):
+    pin(cxx)
+
+
+# (name, original text, mutated text) in ds_oracle.cpp
+MUTATIONS = [
+    ("bf16 shift", "static_cast<uint32_t>(bits) << 16", "static_cast<uint32_t>(bits) << 15"),
+    ("label without the gather", "Kbg[static_cast<int64_t>(t) * d + C[h * r + j]]",
+     "Kbg[static_cast<int64_t>(t) * d + j]"),
+    ("query head to KV head map", "(static_cast<int64_t>(b) * Hkv + h / G) * T * d;\n      uint16_t*",
+     "(static_cast<int64_t>(b) * Hkv + h % Hkv) * T * d;\n      uint16_t*"),
+    ("score uses leading channels of q", "bf16_value(q[C[h * r + j]])", "bf16_value(q[j])"),
+    ("top-k smallest", "return s[a] > s[b];", "return s[a] < s[b];"),
+    ("ties to the higher index", "    return a < b;\n  });", "    return a > b;\n  });"),
+    ("top-k not ascending", "  std::sort(order.begin(), order.begin() + k);\n", ""),
+    ("scale dropped", "l[i] = scale * dot;", "l[i] = dot;"),
+    ("softmax sign", "l[i] = std::exp(l[i] - m);", "l[i] = std::exp(m - l[i]);"),
+    ("softmax not normalised", "const double wi = l[i] / z;", "const double wi = l[i];"),
+    ("lse without max", "  *lse = m + std::log(z);\n}\n\n}  // namespace",
+     "  *lse = std::log(z);\n}\n\n}  // namespace"),
+    ("V rows misaligned with K rows", "V + static_cast<int64_t>(idx[i]) * d",
+     "V + static_cast<int64_t>(idx[(i + 1) % n]) * d"),
+    ("merge weights inverted", "const double a = std::exp(lses[i] - M);",
+     "const double a = std::exp(M - lses[i]);"),
+    ("dense drops the last token", "all[i] = static_cast<int32_t>(i % T);",
+     "all[i] = static_cast<int32_t>(std::min<size_t>(i % T, T - 2));"),
+    ("f32 rounding dropped", "out[i] = static_cast<float>(in[i]);",
+     "out[i] = static_cast<float>(in[i] * (1.0 + 1e-7));"),
+]
+
+
+def _variant(tmp_path, name, old, new):
+    src = open(cxx._SRC).read()
+    assert src.count(old) >= 1, name
+    d = tmp_path / name.replace(" ", "_")
+    d.mkdir()
+    (d / "ds_oracle.cpp").write_text(src.replace(old, new, 1))
+    shutil.copy(os.path.join(os.path.dirname(cxx.__file__), "cxx.py"), d / "cxx.py")
+    spec = importlib.util.spec_from_file_location(f"cxx_mut_{len(os.listdir(tmp_path))}",
+                                                  d / "cxx.py")
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("mut", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_cxx_pins_catch_planted_slip(tmp_path, mut):
+    mod = _variant(tmp_path, *mut)
+    failed = []
+    for pin in pins.CORE_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(mod)
+        except Exception:  # noqa: BLE001  (an assertion, or a bad value further on)
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught: {mut[0]}"
+
+
+@pytest.mark.parametrize("shape", [(2, 4, 4, 300, 16, 20), (2, 8, 2, 257, 8, 33),
+                                   (1, 4, 1, 64, 32, 64)])
+def test_cxx_agrees_with_numpy_oracle(shape):
+    B, Hq, Hkv, T, r, k = shape
+    w = dsgen.Workload("cross", B=B, Hq=Hq, Hkv=Hkv, T=T, r=r, k=k, n_out=min(8, r),
+                       seed=0xC0DE + T)
+    Q, K, V = dsgen.qkv(w)
+    C = dsgen.channels(w, r)
+    a = oracle.sparse_step(Q, K, V, C, k, w.scale)
+    b = cxx.sparse_step(Q, K, V, C, k, w.scale)
+    assert np.array_equal(a["label"], b["label"])
+    assert np.allclose(a["s64"], b["s64"], rtol=1e-13, atol=1e-12)
+    # the two fp32 roundings agree wherever the fp64 scores do to the last bit
+    same = a["s64"] == b["s64"]
+    assert np.array_equal(a["s32"][same], b["s32"][same])
+    assert np.array_equal(oracle.topk(b["s32"], k), b["idx"])
+    assert np.allclose(a["O"], b["O"], atol=1e-12) and np.allclose(a["lse"], b["lse"], atol=1e-12)
+    Od, Ld = cxx.dense(Q, K, V, w.scale)
+    Odn, Ldn = oracle.dense(Q, K, V, w.scale)
+    assert np.allclose(Od, Odn, atol=1e-12) and np.allclose(Ld, Ldn, atol=1e-12)
+
+
+def test_cxx_topk_on_ties_agrees_with_numpy_oracle():
+    rng = np.random.default_rng(11)
+    for T in (1, 5, 64, 1000):
+        s = rng.integers(-2, 3, (3, T)).astype(np.float32)
+        s[rng.random((3, T)) < 0.2] = -0.0
+        for k in sorted({1, max(1, T // 7), T}):
+            assert np.array_equal(cxx.topk(s, k), oracle.topk(s, k))
+            assert np.array_equal(cxx.topk(s.astype(np.float64), k),
+                                  oracle.topk(s.astype(np.float64), k))
