@@ -5,7 +5,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 its Python binding) never imports, links or calls it, and shares no code with
 it: the two meet only at the seeded inputs drawn by ``dsgen``.
 
-``oracle.cxx`` is the C++ oracle of steps O1-O5 (ds_oracle.cpp) with the same
-function names; it shares no code with the numpy oracle below.
+``oracle.cxx`` is the C++ oracle (ds_oracle.cpp) with the same function names
+and results; it shares no code with the numpy oracle below.
 """
 from .ds_oracle import *  # noqa: F401,F403

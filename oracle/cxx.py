@@ -1,10 +1,12 @@
-"""The C++ oracle (oracle/ds_oracle.cpp), steps O1-O5 -- TEST INFRASTRUCTURE ONLY.
+"""The C++ oracle (oracle/ds_oracle.cpp) -- TEST INFRASTRUCTURE ONLY.
 
-The same functions, signatures and results as the numpy oracle's label,
-score, top-k, attention, dense, merge and whole-step functions, computed in
-plain C++ (float64, std::sort, std::exp).  This module only converts arrays
-and calls the library; every arithmetic step runs in ds_oracle.cpp.  The
-library is built here with g++ on first use (or by ``build()``).
+The same functions, signatures and results as the numpy oracle: label,
+score, top-k, attention, dense, merge and the whole step (O1-O5), and the
+calibration, group-shared, block and hierarchical selections beside them,
+computed in plain C++ (float64, std::sort, std::exp).  This module only
+converts arrays and calls the library; every arithmetic step runs in
+ds_oracle.cpp.  The library is built here with g++ on first use (or by
+``build()``).
 
 Only ``tests/`` and ``bench.py``'s CPU-baseline leg use it.
 """
@@ -52,11 +54,24 @@ def _load():
                 "dso_dense": [vp, vp, vp, i32, i32, i32, i32, i32, f64, vp, vp],
                 "dso_lse_merge": [vp, vp, i32, i32, vp, vp],
                 "dso_attend_split": [vp, vp, vp, vp, i32, i32, f64, i32, vp, vp],
+                "dso_calib_importance": [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp],
+                "dso_calib_select": [vp, i32, i32, i32, vp],
+                "dso_group_score_f64": [vp, i32, i32, i32, i32, vp],
+                "dso_group_score_f32": [vp, i32, i32, i32, i32, vp],
+                "dso_group_attend": [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f64, vp,
+                                     vp],
+                "dso_block_score_f64": [vp, i64, i32, i32, vp],
+                "dso_block_score_f32": [vp, i64, i32, i32, vp],
+                "dso_block_tokens": [vp, i32, i32, i32, vp],
+                "dso_block_attend": [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f64,
+                                     vp, vp],
+                "dso_hier_topk_f64": [vp, i64, i32, i32, vp],
+                "dso_hier_topk_f32": [vp, i64, i32, i32, vp],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
-                fn.restype = None
+                fn.restype = ctypes.c_int if name == "dso_block_tokens" else None
             _lib = lib
     return _lib
 
@@ -204,3 +219,127 @@ def sparse_step(Q, K, V, C, k: int, scale):
     idx = topk(s32, k)
     O, L = attend(Q, K, V, idx, scale)
     return {"label": lab, "s64": s64, "s32": s32, "idx": idx, "O": O, "lse": L}
+
+
+# ---- offline channel calibration -------------------------------------------------
+
+def calibrate_importance(Qc, K, T: int, Hq: int):
+    """I [Hq, d] float64 from Qc [B, Hq, Nq, d] and K [B, Hkv, T_cap, d] (tokens < T)."""
+    Qc = _c(Qc, np.uint16)
+    K = _c(K, np.uint16)
+    B, _, Nq, d = Qc.shape
+    _, Hkv, T_cap, _ = K.shape
+    I = np.empty((Hq, d), np.float64)
+    _load().dso_calib_importance(_p(Qc), _p(K), B, Hq, Hkv, Nq, T_cap, T, d, _p(I))
+    return I
+
+
+def calibrate_select(I, r: int):
+    I = _c(I, np.float64)
+    Hq, d = I.shape
+    C = np.empty((Hq, r), np.int32)
+    _load().dso_calib_select(_p(I), Hq, d, r, _p(C))
+    return C
+
+
+def calibrate(Qc, K, T: int, Hq: int, r: int):
+    I = calibrate_importance(Qc, K, T, Hq)
+    return calibrate_select(I, r), I
+
+
+# ---- group-shared selection ------------------------------------------------------
+
+def group_score(s, Hkv: int):
+    """sg [B, Hkv, T] in the precision of s [B, Hq, T] (head order)."""
+    s = np.asarray(s)
+    f32 = s.dtype == np.float32
+    s = _c(s, np.float32 if f32 else np.float64)
+    B, Hq, T = s.shape
+    sg = np.empty((B, Hkv, T), s.dtype)
+    fn = _load().dso_group_score_f32 if f32 else _load().dso_group_score_f64
+    fn(_p(s), B, Hq, Hkv, T, _p(sg))
+    return sg
+
+
+def group_attend(Q, K, V, idx_g, scale):
+    Q = _c(Q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    idx_g = _c(idx_g, np.int32)
+    B, Hq, d = Q.shape
+    _, Hkv, T, _ = K.shape
+    k = idx_g.shape[-1]
+    O = np.empty((B, Hq, d), np.float64)
+    L = np.empty((B, Hq), np.float64)
+    _load().dso_group_attend(_p(Q), _p(K), _p(V), _p(idx_g), B, Hq, Hkv, T, d, k, float(scale),
+                             _p(O), _p(L))
+    return O, L
+
+
+def group_sparse_step(Q, K, V, C, k: int, scale):
+    Hq, Hkv = np.asarray(Q).shape[1], np.asarray(K).shape[1]
+    lab = label(K, C, Hq)
+    s64 = score(Q, C, lab)
+    s32 = to_f32(s64)
+    sg64 = group_score(s64, Hkv)
+    sg32 = group_score(s32, Hkv)
+    idx = topk(sg32, k)
+    O, L = group_attend(Q, K, V, idx, scale)
+    return {"label": lab, "s64": s64, "sg64": sg64, "sg32": sg32, "idx": idx, "O": O, "lse": L}
+
+
+# ---- block-granular selection ----------------------------------------------------
+
+def block_score(s, bs: int):
+    s = np.asarray(s)
+    f32 = s.dtype == np.float32
+    T = s.shape[-1]
+    flat = _c(s.reshape(-1, T), np.float32 if f32 else np.float64)
+    nb = -(-T // bs)
+    out = np.empty((flat.shape[0], nb), flat.dtype)
+    fn = _load().dso_block_score_f32 if f32 else _load().dso_block_score_f64
+    fn(_p(flat), flat.shape[0], T, bs, _p(out))
+    return out.reshape(*s.shape[:-1], nb)
+
+
+def block_tokens(bidx, bs: int, T: int):
+    b = _c(bidx, np.int32)
+    out = np.empty(b.size * bs, np.int32)
+    n = _load().dso_block_tokens(_p(b), b.size, bs, T, _p(out))
+    return out[:n].copy()
+
+
+def block_sparse_step(Q, K, V, C, bs: int, kb: int, scale):
+    Q = _c(Q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    B, Hq, d = Q.shape
+    _, Hkv, T, _ = K.shape
+    lab = label(K, C, Hq)
+    s32 = to_f32(score(Q, C, lab))
+    sb = block_score(s32, bs)
+    bidx = topk(sb, kb)
+    O = np.empty((B, Hq, d), np.float64)
+    L = np.empty((B, Hq), np.float64)
+    _load().dso_block_attend(_p(Q), _p(K), _p(V), _p(bidx), B, Hq, Hkv, T, d, kb, bs,
+                             float(scale), _p(O), _p(L))
+    return {"s32": s32, "sb": sb, "bidx": bidx, "O": O, "lse": L}
+
+
+# ---- hierarchical top-k ------------------------------------------------------------
+
+def hier_topk(s, k: int):
+    s = np.asarray(s)
+    T = s.shape[-1]
+    if not 1 <= k <= T:
+        raise ValueError("need 1 <= k <= T")
+    f32 = s.dtype == np.float32
+    flat = _c(s.reshape(-1, T), np.float32 if f32 else np.float64)
+    out = np.empty((flat.shape[0], k), np.int32)
+    fn = _load().dso_hier_topk_f32 if f32 else _load().dso_hier_topk_f64
+    fn(_p(flat), flat.shape[0], T, k, _p(out))
+    return out.reshape(*s.shape[:-1], k)
+
+
+def hier_topk_head(s, k: int):
+    return hier_topk(np.asarray(s)[None], k)[0]

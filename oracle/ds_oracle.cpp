@@ -1,6 +1,8 @@
 // Plain C++ oracle of Double-Sparsity-style decode attention, steps O1-O5:
 // label gather, channel-sparse score, top-k, softmax attention over the kept
-// rows, dense attention; plus the log-sum-exp merge of split attention.
+// rows, dense attention; plus the log-sum-exp merge of split attention, and the
+// rows beside the path: offline channel calibration, group-shared selection,
+// block-granular selection and the hierarchical top-k.
 //
 // TEST INFRASTRUCTURE ONLY: loaded by tests/ (through oracle/cxx.py) and by
 // the CPU-baseline leg of bench.py, never by the library.  It shares no code
@@ -23,6 +25,22 @@
 //           o = sum_i w_i V_i; lse = m + log sum exp(l - m)
 //   dense   attend with every token kept
 //   merge   disjoint key chunks (o_c, lse_c) combine with weights exp(lse_c - M)
+// and for the rows beside the path (readings shared with oracle/ds_oracle.py):
+//   calibration  I[h,c] = mean over (calibration query n, token t < T) of the
+//                same sequence of |q[b,h,n,c] * k[b,g(h),t,c]|; the r channels
+//                of largest I (ties to the lower channel), ascending.  The
+//                page leaves the criterion open (Method details: Key design).
+//   group        sg[b,g,t] = sum of s[b,h,t] over the query heads h of KV group
+//                g, in head order and in the scores' own precision; one top-k
+//                per group; every head of the group attends over its set
+//   block        (Jenga: Core method 1; Observation 2) per block of bs
+//                consecutive tokens the largest max(s_t, 0); top-kb blocks;
+//                attention over their tokens, clipped to T
+//   hierarchy    (HiP: Core idea, Technical framework) k contiguous parts of
+//                [0, T); while a part is longer than one token, each such part
+//                splits at its middle (the first half one longer), the children
+//                are ranked by the score of their first token (ties to the lower
+//                start) and the first k are kept; the k starts are the result
 //
 // Every value is decoded exactly from its bf16 bits and every step runs in
 // double precision (std::exp, std::log); the order of the top-k is decided by
@@ -84,6 +102,60 @@ void attend_row(const uint16_t* q, const uint16_t* K, const uint16_t* V, const i
     for (int c = 0; c < d; ++c) o[c] += wi * bf16_value(vrow[c]);
   }
   *lse = m + std::log(z);
+}
+
+// Per block of bs tokens the largest max(s_t, 0), for rows of T scores.
+template <class S>
+void block_score_rows(const S* s, int64_t rows, int T, int bs, S* sb) {
+  const int nb = (T + bs - 1) / bs;
+  for (int64_t i = 0; i < rows; ++i)
+    for (int j = 0; j < nb; ++j) {
+      S m = 0;
+      for (int t = j * bs; t < std::min((j + 1) * bs, T); ++t) m = std::max(m, s[i * T + t]);
+      sb[i * nb + j] = m;
+    }
+}
+
+// Ascending token ids of the blocks bidx[0..kb) of bs tokens each, clipped to
+// T; returns their number.
+int block_tokens_row(const int32_t* bidx, int kb, int bs, int T, int32_t* out) {
+  std::vector<int32_t> blocks(bidx, bidx + kb);
+  std::sort(blocks.begin(), blocks.end());
+  int n = 0;
+  for (int32_t j : blocks)
+    for (int t = j * bs; t < std::min((j + 1) * bs, T); ++t) out[n++] = t;
+  return n;
+}
+
+// The hierarchical search over one head's scores s[0..T) keeping k tokens.
+template <class S>
+void hier_row(const S* s, int T, int k, int32_t* out) {
+  std::vector<std::pair<int, int>> parts;  // [begin, end)
+  for (int i = 0; i < k; ++i)
+    parts.emplace_back(static_cast<int>(static_cast<int64_t>(i) * T / k),
+                       static_cast<int>(static_cast<int64_t>(i + 1) * T / k));
+  auto longer = [](const std::pair<int, int>& p) { return p.second - p.first > 1; };
+  while (std::any_of(parts.begin(), parts.end(), longer)) {
+    std::vector<std::pair<int, int>> children;
+    for (const auto& p : parts) {
+      if (longer(p)) {
+        const int m = p.first + (p.second - p.first + 1) / 2;
+        children.emplace_back(p.first, m);
+        children.emplace_back(m, p.second);
+      } else {
+        children.push_back(p);
+      }
+    }
+    std::sort(children.begin(), children.end(),
+              [s](const std::pair<int, int>& a, const std::pair<int, int>& b) {
+                if (s[a.first] != s[b.first]) return s[a.first] > s[b.first];
+                return a.first < b.first;
+              });
+    children.resize(k);
+    std::sort(children.begin(), children.end());
+    parts = children;
+  }
+  for (int i = 0; i < k; ++i) out[i] = parts[i].first;
 }
 
 }  // namespace
@@ -194,6 +266,118 @@ void dso_attend_split(const uint16_t* q, const uint16_t* K, const uint16_t* V,
     start += len;
   }
   dso_lse_merge(outs.data(), lses.data(), static_cast<int>(lses.size()), d, o, lse);
+}
+
+// Calibration importance.  Qc [B, Hq, Nq, d], K [B, Hkv, T_cap, d] (tokens
+// 0..T-1) -> I [Hq, d].  |q k| = |q| |k|, so per sequence the double sum over
+// (n, t) is the product of the two single sums.
+void dso_calib_importance(const uint16_t* Qc, const uint16_t* K, int B, int Hq, int Hkv, int Nq,
+                          int T_cap, int T, int d, double* I) {
+  const int G = Hq / Hkv;
+  for (int i = 0; i < Hq * d; ++i) I[i] = 0.0;
+  std::vector<double> ksum(static_cast<size_t>(Hkv) * d), qsum(d);
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g)
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int t = 0; t < T; ++t) {
+          const int64_t row = (static_cast<int64_t>(b) * Hkv + g) * T_cap + t;
+          acc += std::fabs(bf16_value(K[row * d + c]));
+        }
+        ksum[static_cast<size_t>(g) * d + c] = acc;
+      }
+    for (int h = 0; h < Hq; ++h) {
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int n = 0; n < Nq; ++n)
+          acc += std::fabs(bf16_value(Qc[((static_cast<int64_t>(b) * Hq + h) * Nq + n) * d + c]));
+        qsum[c] = acc;
+      }
+      const double* kg = ksum.data() + static_cast<size_t>(h / G) * d;
+      for (int c = 0; c < d; ++c) I[h * d + c] += qsum[c] * kg[c];
+    }
+  }
+  const double n = static_cast<double>(B) * Nq * T;
+  for (int i = 0; i < Hq * d; ++i) I[i] /= n;
+}
+
+// Calibration choice: I [Hq, d] -> C [Hq, r], the r channels of largest
+// importance (ties to the lower channel), ascending.
+void dso_calib_select(const double* I, int Hq, int d, int r, int32_t* C) {
+  dso_topk_f64(I, Hq, d, r, C);
+}
+
+// Group scores: s [B, Hq, T] -> sg [B, Hkv, T], the member heads' scores added
+// in head order, in the scores' own precision.
+void dso_group_score_f64(const double* s, int B, int Hq, int Hkv, int T, double* sg) {
+  const int G = Hq / Hkv;
+  for (int64_t i = 0; i < static_cast<int64_t>(B) * Hkv * T; ++i) sg[i] = 0.0;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hq; ++h)
+      for (int t = 0; t < T; ++t)
+        sg[(static_cast<int64_t>(b) * Hkv + h / G) * T + t] +=
+            s[(static_cast<int64_t>(b) * Hq + h) * T + t];
+}
+void dso_group_score_f32(const float* s, int B, int Hq, int Hkv, int T, float* sg) {
+  const int G = Hq / Hkv;
+  for (int64_t i = 0; i < static_cast<int64_t>(B) * Hkv * T; ++i) sg[i] = 0.0f;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hq; ++h)
+      for (int t = 0; t < T; ++t)
+        sg[(static_cast<int64_t>(b) * Hkv + h / G) * T + t] +=
+            s[(static_cast<int64_t>(b) * Hq + h) * T + t];
+}
+
+// Group attention: query head h attends over its group's set idx_g [B, Hkv, k].
+void dso_group_attend(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                      const int32_t* idx_g, int B, int Hq, int Hkv, int T, int d, int k,
+                      double scale, double* O, double* lse) {
+  const int G = Hq / Hkv;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hq; ++h) {
+      const int64_t bh = static_cast<int64_t>(b) * Hq + h;
+      const int64_t bg = static_cast<int64_t>(b) * Hkv + h / G;
+      attend_row(Q + bh * d, K + bg * T * d, V + bg * T * d, idx_g + bg * k, k, d, scale,
+                 O + bh * d, lse + bh, nullptr);
+    }
+}
+
+// Block scores: s [rows, T] -> sb [rows, ceil(T / bs)], per block the largest
+// max(s_t, 0) (the last block may be short).
+void dso_block_score_f64(const double* s, int64_t rows, int T, int bs, double* sb) {
+  block_score_rows(s, rows, T, bs, sb);
+}
+void dso_block_score_f32(const float* s, int64_t rows, int T, int bs, float* sb) {
+  block_score_rows(s, rows, T, bs, sb);
+}
+
+// Token ids of one head's blocks (ascending, clipped to T); returns the count.
+int dso_block_tokens(const int32_t* bidx, int kb, int bs, int T, int32_t* out) {
+  return block_tokens_row(bidx, kb, bs, T, out);
+}
+
+// Block attention: each head over the tokens of its blocks bidx [B, Hq, kb].
+void dso_block_attend(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                      const int32_t* bidx, int B, int Hq, int Hkv, int T, int d, int kb, int bs,
+                      double scale, double* O, double* lse) {
+  const int G = Hq / Hkv;
+  std::vector<int32_t> toks(static_cast<size_t>(kb) * bs);
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hq; ++h) {
+      const int64_t bh = static_cast<int64_t>(b) * Hq + h;
+      const int64_t bg = static_cast<int64_t>(b) * Hkv + h / G;
+      const int n = block_tokens_row(bidx + bh * kb, kb, bs, T, toks.data());
+      attend_row(Q + bh * d, K + bg * T * d, V + bg * T * d, toks.data(), n, d, scale,
+                 O + bh * d, lse + bh, nullptr);
+    }
+}
+
+// Hierarchical top-k: s [rows, T] -> idx [rows, k]; 1 <= k <= T.
+void dso_hier_topk_f64(const double* s, int64_t rows, int T, int k, int32_t* idx) {
+  for (int64_t i = 0; i < rows; ++i) hier_row(s + i * T, T, k, idx + i * k);
+}
+void dso_hier_topk_f32(const float* s, int64_t rows, int T, int k, int32_t* idx) {
+  for (int64_t i = 0; i < rows; ++i) hier_row(s + i * T, T, k, idx + i * k);
 }
 
 }  // extern "C"

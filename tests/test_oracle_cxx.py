@@ -1,11 +1,12 @@
-"""The C++ oracle (steps O1-O5 and the merge, oracle/ds_oracle.cpp), no GPU needed.
+"""The C++ oracle (oracle/ds_oracle.cpp), no GPU needed.
 
-1. The same pins as the numpy oracle's steps: bf16 decoding, label gather,
-   score, top-k order and worked examples, attention against torch's
-   scaled_dot_product_attention and closed forms, merge invariance, dense,
-   r = d with k = T.
+1. Every pin of the numpy oracle, run against the C++ one: bf16 decoding,
+   label gather, score, top-k order and worked examples, attention against
+   torch's scaled_dot_product_attention and closed forms, merge invariance,
+   dense, r = d with k = T; calibration, group-shared, block and hierarchical
+   selection.
 2. Planted slips in a copy of the C++ source (compiled into a temporary
-   directory): each must make at least one of those pins fail.
+   directory): each must make at least one pin fail.
 3. Agreement with the numpy oracle on seeded workloads (MHA and grouped KV
    heads, tie-heavy scores): the two implementations share no code.
 """
@@ -22,7 +23,7 @@ import oracle.cxx as cxx
 from tests import pins
 
 
-@pytest.mark.parametrize("pin", pins.CORE_PINS, ids=lambda p: p.__name__)
+@pytest.mark.parametrize("pin", pins.PINS, ids=lambda p: p.__name__)
 def test_cxx_pin(pin):
     pin(cxx)
 
@@ -41,8 +42,7 @@ MUTATIONS = [
     ("scale dropped", "l[i] = scale * dot;", "l[i] = dot;"),
     ("softmax sign", "l[i] = std::exp(l[i] - m);", "l[i] = std::exp(m - l[i]);"),
     ("softmax not normalised", "const double wi = l[i] / z;", "const double wi = l[i];"),
-    ("lse without max", "  *lse = m + std::log(z);\n}\n\n}  // namespace",
-     "  *lse = std::log(z);\n}\n\n}  // namespace"),
+    ("lse without max", "*lse = m + std::log(z);", "*lse = std::log(z);"),
     ("V rows misaligned with K rows", "V + static_cast<int64_t>(idx[i]) * d",
      "V + static_cast<int64_t>(idx[(i + 1) % n]) * d"),
     ("merge weights inverted", "const double a = std::exp(lses[i] - M);",
@@ -51,6 +51,31 @@ MUTATIONS = [
      "all[i] = static_cast<int32_t>(std::min<size_t>(i % T, T - 2));"),
     ("f32 rounding dropped", "out[i] = static_cast<float>(in[i]);",
      "out[i] = static_cast<float>(in[i] * (1.0 + 1e-7));"),
+    ("calibration without magnitudes", "acc += std::fabs(bf16_value(K[row * d + c]));",
+     "acc += bf16_value(K[row * d + c]);"),
+    ("calibration reads past T", "for (int t = 0; t < T; ++t) {\n          const int64_t row",
+     "for (int t = 0; t < T_cap; ++t) {\n          const int64_t row"),
+    ("calibration sums q and k", "I[h * d + c] += qsum[c] * kg[c];",
+     "I[h * d + c] += qsum[c] + kg[c];"),
+    ("calibration ignores importance", "dso_topk_f64(I, Hq, d, r, C);",
+     "for (int i = 0; i < Hq * r; ++i) C[i] = i % r;"),
+    ("group score in the wrong group", "sg[(static_cast<int64_t>(b) * Hkv + h / G) * T + t] +=",
+     "sg[(static_cast<int64_t>(b) * Hkv + h % Hkv) * T + t] +="),
+    ("group attention on the wrong group",
+     "const int64_t bg = static_cast<int64_t>(b) * Hkv + h / G;",
+     "const int64_t bg = static_cast<int64_t>(b) * Hkv + h % Hkv;"),
+    ("block score keeps negatives", "      S m = 0;\n", "      S m = s[i * T + j * bs];\n"),
+    ("block tokens off by one", "for (int t = j * bs; t < std::min((j + 1) * bs, T); ++t) out",
+     "for (int t = j * bs + 1; t < std::min((j + 1) * bs, T); ++t) out"),
+    ("hierarchy halves the other way", "const int m = p.first + (p.second - p.first + 1) / 2;",
+     "const int m = p.first + (p.second - p.first) / 2;"),
+    ("hierarchy ties to the higher start", "return a.first < b.first;",
+     "return a.first > b.first;"),
+    ("hierarchy keeps the worst parts", "return s[a.first] > s[b.first];",
+     "return s[a.first] < s[b.first];"),
+    ("hierarchy scores parts by their last token",
+     "if (s[a.first] != s[b.first]) return s[a.first] > s[b.first];",
+     "if (s[a.second - 1] != s[b.second - 1]) return s[a.second - 1] > s[b.second - 1];"),
 ]
 
 
@@ -72,7 +97,7 @@ def _variant(tmp_path, name, old, new):
 def test_cxx_pins_catch_planted_slip(tmp_path, mut):
     mod = _variant(tmp_path, *mut)
     failed = []
-    for pin in pins.CORE_PINS:
+    for pin in pins.PINS:
         try:
             with np.errstate(all="ignore"):
                 pin(mod)
@@ -112,3 +137,27 @@ def test_cxx_topk_on_ties_agrees_with_numpy_oracle():
             assert np.array_equal(cxx.topk(s, k), oracle.topk(s, k))
             assert np.array_equal(cxx.topk(s.astype(np.float64), k),
                                   oracle.topk(s.astype(np.float64), k))
+
+
+def test_cxx_rows_beside_the_path_agree_with_numpy_oracle():
+    w = dsgen.Workload("cross-next", B=2, Hq=8, Hkv=2, T=300, r=16, k=24, n_out=8,
+                       seed=0xC0DF)
+    Q, K, V = dsgen.qkv(w)
+    C = dsgen.channels(w, 16)
+    Qc = dsgen.q_calib(w, 5)
+    Ca, Ia = oracle.calibrate(Qc, K, 290, w.Hq, 8)
+    Cb, Ib = cxx.calibrate(Qc, K, 290, w.Hq, 8)
+    assert np.array_equal(Ca, Cb) and np.allclose(Ia, Ib, rtol=1e-13, atol=0)
+    a = oracle.group_sparse_step(Q, K, V, C, w.k, w.scale)
+    b = cxx.group_sparse_step(Q, K, V, C, w.k, w.scale)
+    assert np.array_equal(a["sg32"], b["sg32"]) and np.array_equal(a["idx"], b["idx"])
+    assert np.allclose(a["sg64"], b["sg64"], rtol=1e-13, atol=1e-12)
+    assert np.allclose(a["O"], b["O"], atol=1e-12) and np.allclose(a["lse"], b["lse"], atol=1e-12)
+    for bs, kb in ((64, 2), (7, 5), (1, 9)):
+        a = oracle.block_sparse_step(Q, K, V, C, bs, kb, w.scale)
+        b = cxx.block_sparse_step(Q, K, V, C, bs, kb, w.scale)
+        assert np.array_equal(a["sb"], b["sb"]) and np.array_equal(a["bidx"], b["bidx"])
+        assert np.allclose(a["O"], b["O"], atol=1e-12)
+    s32 = cxx.sparse_step(Q, K, V, C, w.k, w.scale)["s32"]
+    for k in (1, 5, 24, 300):
+        assert np.array_equal(oracle.hier_topk(s32, k), cxx.hier_topk(s32, k))
