@@ -40,9 +40,11 @@
  *     ds_label_append (Double Sparsity page, Abstract and Experimental
  *     highlights: combined with offloading the KV cache to host memory).
  *     Other host memory is refused with DS_ERR_INVALID_ARG before launch.
- *     ds_decode_step also takes Q, O and lse in such host memory: a decode
- *     loop then hands the step its query and reads its result with no copy
- *     of their own (the kernel reads Q and writes O over the host link).
+ *     ds_decode_step and ds_decode_step_kv also take Q, O and lse (and
+ *     ds_decode_step_kv its new K/V rows, as ds_kv_append does) in such host
+ *     memory: a decode loop then hands the step its query and reads its
+ *     result with no copy of their own (the kernel reads Q and writes O over
+ *     the host link).
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns DS_ERR_INVALID_ARG (or DS_ERR_UNSUPPORTED for a valid
  *     but unimplemented shape) and launches nothing.
