@@ -12,7 +12,7 @@
  *   B      sequences in the batch
  *   Hq     query heads; Hkv KV heads; Hq % Hkv == 0; query head h reads
  *          KV head g(h) = h / (Hq / Hkv)
- *   d      head dimension; this build supports d == 128 only
+ *   d      head dimension; the library supports d == 128 only
  *   T_cap  token capacity of the K/V and label caches; T <= T_cap tokens valid
  *   r      label channels per query head (1 <= r <= d)
  *   k      tokens kept per query head (1 <= k <= T)

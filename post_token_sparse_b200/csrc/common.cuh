@@ -6,7 +6,7 @@
 
 namespace ds {
 
-constexpr int kHeadDim = 128;          // d: the only head size this build supports
+constexpr int kHeadDim = 128;          // d: the only head size the library supports
 constexpr int kRowBytes = kHeadDim * 2; // one bf16 K or V row
 
 // Per-device status word: kernels OR bits into it instead of faulting.
