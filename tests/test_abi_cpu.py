@@ -295,3 +295,37 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
                          cwd=tmp_path, capture_output=True, text=True)
     assert res.returncode != 0
     assert "libds.so is missing" in res.stderr
+
+
+def _plan(heads, rows, sparse):
+    """The documented split rule: at most 2048 rows per sparse split, at least 64
+    rows, the smallest split count whose grid fills its last wave of 148 x 6 CTAs
+    to within 10% (else the best filled), rows per split a multiple of 4."""
+    import math
+    wave = 148 * 6
+    s_min = -(-rows // 2048) if sparse else 1
+    s_max = max(s_min, min(256, rows // 64))
+    best, best_waste = s_min, math.inf
+    for S in range(s_min, s_max + 1):
+        n = heads * S
+        waste = math.ceil(n / wave) * wave / n
+        if waste < best_waste - 1e-9:
+            best, best_waste = S, waste
+        if waste <= 1.10:
+            break
+    rps = -(-rows // best)
+    rps = (rps + 3) & ~3
+    return -(-rows // rps)
+
+
+@pytest.mark.parametrize("B,H,T,k", [(1, 32, 262144, 16384), (32, 32, 32768, 512),
+                                     (32, 32, 32768, 2048), (8, 32, 4096, 256),
+                                     (16, 64, 16384, 1024), (1, 4, 1000, 1000),
+                                     (3, 7, 5000, 300), (1, 1, 300000, 4000)])
+def test_split_plan_follows_the_documented_rule(B, H, T, k):
+    lib = ds.lib()
+    d = _dims(B=B, Hq=H, Hkv=H, T_cap=T, r=8)
+    for op, rows, sparse in ((ds.OP_SPARSE_DECODE, k, True), (ds.OP_DECODE, T, False)):
+        S = _plan(B * H, rows, sparse)
+        want = 0 if S <= 1 else (B * H * S * 132 * 4 + B * H * 4 + 255) // 256 * 256
+        assert lib.ds_workspace_size(op, d, T, k if sparse else T) == want, (op, S)
