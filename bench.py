@@ -847,7 +847,10 @@ def main():
         dn = dense_entry(w, max(20, args.steps // 10), 3, hbm_peak, inputs=inputs)
         line["dense"] = dn
         line["speedup_vs_dense"] = dn["us_per_step"] / line["us_per_step"]
-        line["cpu_baseline"] = time_oracle(base, args.cpu_seconds)
+        try:
+            line["cpu_baseline"] = time_oracle(base, args.cpu_seconds)
+        except Exception as e:  # noqa: BLE001  (the GPU figures stand without it)
+            line["cpu_baseline"] = {"kind": "oracle", "error": repr(e)[:200]}
         line["calibrate"] = _rounded(calib_entry(w, inputs[1], hbm_peak))
         line["block_select"] = _rounded(block_entry(w, inputs, hbm_peak))
         line["hier_select"] = _rounded(hier_entry(w, inputs, hbm_peak))
