@@ -391,9 +391,13 @@ def time_e2e(step: Step, steps: int, warmup: int):
 # ---------------------------------------------------------------------------
 # the CPU oracle, timed on a bounded sample of heads
 
-def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
+def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False,
+                max_heads: int | None = None):
     """The oracle's score + top-k + attention per head, one thread: the C++ oracle
-    (steps O1-O5), or the numpy oracle where the C++ one cannot be built."""
+    (steps O1-O5), or the numpy oracle where the C++ one cannot be built.  Heads are
+    drawn in a seeded random order until the budget of oracle time is spent (or
+    max_heads heads are done); a workload whose heads all fit is timed over
+    repeated passes."""
     import numpy as np
 
     try:
@@ -440,7 +444,7 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False):
         if cached_bytes <= (2 << 30):  # keep the inputs for further passes
             cache.append((q, C[h], lab, Kbg, Vbg))
             cached_bytes += Kbg.nbytes + Vbg.nbytes + lab.nbytes
-        if elapsed + dense_el >= budget_s:
+        if elapsed + dense_el >= budget_s or (max_heads is not None and done >= max_heads):
             break
     passes = 1
     # a short workload is timed over repeated passes (inputs kept), up to the budget
@@ -746,6 +750,10 @@ def run_sweep(skip: str, hbm_peak: float):
             e["kv_offload"] = offload_entry(ww, hbm_peak)
         if ww.k <= 2048 and (first_of_set or ww.Hq > ww.Hkv) and ww.T > 4096:
             e["hier_select"] = hier_entry(ww, inp, hbm_peak, steps=20)
+        try:  # the oracle on the host cores beside each workload: a few heads
+            e["cpu_baseline"] = time_oracle(ww, 1.0, max_heads=8 if ww.T <= 32768 else 3)
+        except Exception as ex:  # noqa: BLE001  (the GPU figures stand without it)
+            e["cpu_baseline"] = {"kind": "oracle", "error": repr(ex)[:200]}
         out[name] = _rounded(e)
         if name == dsgen.ORDER[-1] and name.startswith("sweep"):
             full = ww.with_(name="sweep-B32-H32-T32K-r128-kT", r=ww.d, k=ww.T)

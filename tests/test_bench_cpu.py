@@ -68,3 +68,9 @@ def test_traffic_profile_used_only_for_the_profiled_sources(tmp_path, monkeypatc
     assert bench.profiled_traffic("k_step") is None
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(tmp_path / "missing.txt"))
     assert bench.profiled_traffic("k_step") is None
+
+
+def test_cpu_baseline_head_cap():
+    r = bench.time_oracle(dsgen.workload("sweep-B32-H32-T32K-r8-k512"), 30.0, max_heads=2)
+    assert r["sample"].startswith("2 head-steps") and r["value"] > 0
+    assert r["us_per_step"] > 0 and r["cores"] == 1
