@@ -70,6 +70,9 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--batch", type=int, default=None,
                    help="override the workload's batch size (smaller captures for ncu)")
+    p.add_argument("--summarize-ncu", metavar="DIR", default=None,
+                   help="no GPU: write the profiles/ summaries from DIR/launches.csv and "
+                        "DIR/k_step_headline.ncu-rep (the ncu runs of the small command)")
     return p.parse_args()
 
 
@@ -763,8 +766,124 @@ def run_sweep(skip: str, hbm_peak: float):
     return out
 
 
+# ---------------------------------------------------------------------------
+# profiles/: text summaries of the ncu runs of the small bench command
+
+SMALL_CMD = "python bench.py --steps 20 --warmup 5 --no-sweep --cpu-seconds 1"
+
+
+def summarize_ncu(src: str) -> None:
+    """Write profiles/ from an ncu launch list (src/launches.csv, made by
+    ``ncu --metrics gpu__time_duration.sum --clock-control none --csv --log-file
+    launches.csv <SMALL_CMD>``) and a full capture of the step kernel
+    (src/k_step_headline.ncu-rep, ``ncu --set full --clock-control none -k
+    regex:k_step -s 5 -c 1 -o k_step_headline <SMALL_CMD>``), read with ``ncu -i``."""
+    import collections
+    import csv
+    import io
+    import re
+    import subprocess
+
+    w = dsgen.workload(HEADLINE)
+    shape = f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} r={w.r} k={w.k}"
+    prof = os.path.join(ROOT, "profiles")
+    made = "# command (one B200; the same command exited 0 without ncu first, in the same call):"
+    # launch list: launches, total time and share per kernel
+    rows = [r for r in csv.reader(open(os.path.join(src, "launches.csv"))) if len(r) > 10]
+    ki, vi = rows[0].index("Kernel Name"), rows[0].index("Metric Value")
+    agg = collections.OrderedDict()
+    for r in rows[1:]:
+        a = agg.setdefault(re.sub(r"\(.*", "", r[ki]).replace("void ", ""), [0, 0.0])
+        a[0] += 1
+        a[1] += float(r[vi]) / 1e3
+    tot = sum(v[1] for v in agg.values())
+    ours = sum(v[1] for k, v in agg.items() if k.startswith("ds::"))
+    lines = [f"# Launch list of the small bench run, workload {w.name} ({shape})", made,
+             "#   ncu --metrics gpu__time_duration.sum --clock-control none --csv --log-file "
+             "launches.csv \\", f"#       {SMALL_CMD}",
+             f"# summarised by: python bench.py --summarize-ncu <dir of the ncu outputs>",
+             "# Under ncu every launch runs serialised with cold caches: compare shares, not "
+             "absolute times.",
+             "# at::...FillFunctor<unsigned char> is the bench's 256 MiB L2 flush between timed "
+             "steps (outside",
+             "# the timed region); the other at:: kernels are setup.  Shares of the library's own "
+             "kernels are",
+             "# also given relative to their sum.", "",
+             f"{'kernel':58s} {'launches':>8s} {'total us':>11s} {'share':>7s} {'share(ds)':>9s} "
+             f"{'avg us':>8s}"]
+    for k, (n, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
+        sd = f"{100 * t / ours:8.1f}%" if k.startswith("ds::") else " " * 9
+        lines.append(f"{k[:58]:58s} {n:8d} {t:11.1f} {100 * t / tot:6.1f}% {sd} {t / n:8.2f}")
+    lines.append(f"{'total':58s} {len(rows) - 1:8d} {tot:11.1f}")
+    open(os.path.join(prof, f"launches_{w.name}.txt"), "w").write("\n".join(lines) + "\n")
+
+    # the step kernel's full capture
+    raw = subprocess.run(["ncu", "-i", os.path.join(src, "k_step_headline.ncu-rep"), "--page",
+                          "raw", "--csv"], capture_output=True, text=True, check=True).stdout
+    rr = list(csv.reader(io.StringIO(raw)))
+    h, units, vals = rr[0], rr[1], rr[2]
+
+    def get(m):
+        return (vals[h.index(m)], units[h.index(m)]) if m in h else ("n/a", "")
+
+    def num(m):
+        v, u = get(m)
+        return float(v.replace(",", "")) * {"Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(u, 1)
+
+    rd, wr = num("dram__bytes_read.sum"), num("dram__bytes_write.sum")
+    dur = num("gpu__time_duration.sum") / (1e3 if get("gpu__time_duration.sum")[1] == "ns"
+                                           else 1)
+    alg = stage_bytes(w)["decode_step"]
+    pre, post = "smsp__average_warps_issue_stalled_", "_per_issue_active.ratio"
+    stalls = sorted(((float(vals[i] or 0), m[len(pre):-len(post)]) for i, m in enumerate(h)
+                     if m.startswith(pre) and m.endswith(post) and float(vals[i] or 0) >= 0.05),
+                    reverse=True)
+    cmd = f"ncu --set full --clock-control none -k regex:k_step -s 5 -c 1 -o k_step_headline " \
+          f"{SMALL_CMD}"
+    L = [f"# k_step<{w.r}> (ds_decode_step, one launch per decode step), workload {w.name}", made,
+         f"#   {cmd}", "# summarised by: python bench.py --summarize-ncu <dir of the ncu outputs>",
+         "# the 6th k_step launch (a graph-replayed timed step); ncu flushes caches before it "
+         "(cold).",
+         f"duration_us (under ncu, cold): {dur:.2f}",
+         f"dram_bytes_read: {rd:.0f}", f"dram_bytes_write: {wr:.0f}",
+         f"dram_bytes_total: {rd + wr:.0f}",
+         f"algorithmic_bytes_per_launch: {alg}  (labels + selected K/V rows + idx + Q/O + new "
+         "label rows)",
+         f"traffic / algorithmic: {(rd + wr) / alg:.3f}",
+         "dram throughput (% of peak, elapsed): "
+         f"{get('gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed')[0]}",
+         "sm throughput (% of peak, elapsed): "
+         f"{get('sm__throughput.avg.pct_of_peak_sustained_elapsed')[0]}",
+         "issue active (% of active cycles): "
+         f"{get('smsp__issue_active.avg.pct_of_peak_sustained_active')[0]}",
+         f"registers/thread: {get('launch__registers_per_thread')[0]}  grid: "
+         f"{get('launch__grid_size')[0]}  block: {get('launch__block_size')[0]}",
+         f"dynamic smem/block: {get('launch__shared_mem_per_block_dynamic')[0]} "
+         f"{get('launch__shared_mem_per_block_dynamic')[1]}",
+         f"occupancy limit (registers): {get('launch__occupancy_limit_registers')[0]} blocks/SM",
+         "warps active (% of peak, active cycles): "
+         f"{get('sm__warps_active.avg.pct_of_peak_sustained_active')[0]}",
+         f"L2 hit rate (%): {get('lts__t_sector_hit_rate.pct')[0]}",
+         "shared-memory bank conflicts (sum): "
+         f"{get('l1tex__data_bank_conflicts_pipe_lsu_mem_shared.sum')[0]}",
+         "warp stall reasons (cycles per issued instruction, >= 0.05):"]
+    L += [f"  {n:24s} {v:.2f}" for v, n in stalls]
+    open(os.path.join(prof, f"k_step_{w.name}.txt"), "w").write("\n".join(L) + "\n")
+
+    T = [f"# DRAM traffic per launch of the dominant kernel, workload {w.name} ({shape})",
+         f"# from the full capture summarised in profiles/k_step_{w.name}.txt:", f"#   {cmd}",
+         "# read by bench.py for roofline.traffic while kernel_source_hash matches the sources.",
+         f"kernel_source_hash: {kernel_source_hash()}",
+         f"dram_bytes_per_launch[k_step]: {rd + wr:.0f}",
+         f"gpu_time_ns[k_step]: {dur * 1e3:.0f}"]
+    open(os.path.join(prof, f"traffic_{w.name}.txt"), "w").write("\n".join(T) + "\n")
+
+
 def main():
     args = parse()
+    if args.summarize_ncu:
+        summarize_ncu(args.summarize_ncu)
+        return 0
     rank, local_rank, world = rank_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
