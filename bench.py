@@ -279,9 +279,10 @@ class Step:
     def replay(self):
         self.graph.replay()
 
-    def timed(self):
-        """One step after an L2 flush: (step ms, [stage ms])."""
-        flush_l2(self.flush)
+    def timed(self, flush: bool = True):
+        """One step after an L2 flush (or without one): (step ms, [stage ms])."""
+        if flush:
+            flush_l2(self.flush)
         self.graph.replay()
         self.torch.cuda.synchronize()
         ev = self.events
@@ -396,20 +397,23 @@ def time_e2e(step: Step, steps: int, warmup: int):
 
 def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False,
                 max_heads: int | None = None):
-    """The oracle's score + top-k + attention per head, one thread: the C++ oracle
-    (steps O1-O5), or the numpy oracle where the C++ one cannot be built.  Heads are
+    """Both oracles' score + top-k + attention per head, one thread each, on the same
+    heads: the numpy oracle and the C++ one (when it can be built).  The faster is
+    reported (the conservative baseline), the other's rate beside it.  Heads are
     drawn in a seeded random order until the budget of oracle time is spent (or
     max_heads heads are done); a workload whose heads all fit is timed over
     repeated passes."""
     import numpy as np
 
+    import oracle as orc_np
+
+    impls = {"float64 numpy": orc_np}
     try:
-        import oracle.cxx as oracle
-        oracle.build()
-        kind = "float64 C++ (std::sort, std::exp)"
-    except Exception:  # noqa: BLE001  (no C++ compiler: the numpy oracle, said so)
-        import oracle
-        kind = "float64 numpy"
+        import oracle.cxx as orc_cxx
+        orc_cxx.build()
+        impls["float64 C++ (std::sort, std::exp)"] = orc_cxx
+    except Exception:  # noqa: BLE001  (no C++ compiler: numpy alone, said so)
+        pass
 
     try:
         from threadpoolctl import threadpool_limits
@@ -420,20 +424,25 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False,
     order = rng.permutation(w.B * w.Hq)
     C = dsgen.channels(w)
     per_head = w.T * w.r * 2 + w.k * 4 * w.d + w.d * 6
-    done, elapsed, dense_el = 0, 0.0, 0.0
+    done = 0
+    elapsed = {n: 0.0 for n in impls}
+    dense_el = {n: 0.0 for n in impls}
     cache, cached_bytes, passes = [], 0, 0
 
+    def spent():
+        return sum(elapsed.values()) + sum(dense_el.values())
+
     def run_head(q, Ch, lab, Kbg, Vbg):
-        nonlocal elapsed, dense_el
-        t0 = time.perf_counter()
-        s = oracle.to_f32(oracle.score_head(q, Ch, lab))
-        idx = oracle.topk_head(s, w.k)
-        oracle.attend_head(q, Kbg, Vbg, idx, w.scale)
-        elapsed += time.perf_counter() - t0
-        if with_dense:
+        for n, orc in impls.items():
             t0 = time.perf_counter()
-            oracle.attend_head(q, Kbg, Vbg, np.arange(w.T), w.scale)
-            dense_el += time.perf_counter() - t0
+            s = orc.to_f32(orc.score_head(q, Ch, lab))
+            idx = orc.topk_head(s, w.k)
+            orc.attend_head(q, Kbg, Vbg, idx, w.scale)
+            elapsed[n] += time.perf_counter() - t0
+            if with_dense:
+                t0 = time.perf_counter()
+                orc.attend_head(q, Kbg, Vbg, np.arange(w.T), w.scale)
+                dense_el[n] += time.perf_counter() - t0
 
     for p in order:
         b, h = divmod(int(p), w.Hq)
@@ -441,31 +450,35 @@ def time_oracle(w: dsgen.Workload, budget_s: float, with_dense: bool = False,
         q = dsgen.q_slab(w, b, h)
         Kbg = dsgen.kv_slab(w, "K", b, g)
         Vbg = dsgen.kv_slab(w, "V", b, g)
-        lab = oracle.label_head(Kbg, C[h])  # label cache: setup, not timed
+        lab = orc_np.label_head(Kbg, C[h])  # label cache: setup, not timed
         run_head(q, C[h], lab, Kbg, Vbg)
         done += 1
         if cached_bytes <= (2 << 30):  # keep the inputs for further passes
             cache.append((q, C[h], lab, Kbg, Vbg))
             cached_bytes += Kbg.nbytes + Vbg.nbytes + lab.nbytes
-        if elapsed + dense_el >= budget_s or (max_heads is not None and done >= max_heads):
+        if spent() >= budget_s or (max_heads is not None and done >= max_heads):
             break
     passes = 1
     # a short workload is timed over repeated passes (inputs kept), up to the budget
-    while len(cache) == w.B * w.Hq and elapsed + dense_el < budget_s and passes < 1000:
+    while len(cache) == w.B * w.Hq and spent() < budget_s and passes < 1000:
         for item in cache:
             run_head(*item)
             done += 1
         passes += 1
     if limit is not None:
         limit.unregister() if hasattr(limit, "unregister") else None
-    us_step = elapsed / done * w.B * w.Hq * 1e6
-    out = {"value": per_head * done / elapsed / 1e9, "unit": "GB/s", "cores": 1,
-           "kind": "oracle", "us_per_step": us_step,
+    rates = {n: per_head * done / elapsed[n] / 1e9 for n in impls}
+    best = max(rates, key=rates.get)
+    others = ", ".join(f"{n}: {v:.3f} GB/s" for n, v in rates.items() if n != best)
+    out = {"value": rates[best], "unit": "GB/s", "cores": 1,
+           "kind": "oracle", "us_per_step": elapsed[best] / done * w.B * w.Hq * 1e6,
            "sample": f"{done} head-steps ({passes} pass(es) over the {w.B * w.Hq} heads) of "
-                     f"{w.name}, score + top-k + attention per head in {kind}, one "
-                     f"thread ({elapsed:.1f} s)"}
+                     f"{w.name}, score + top-k + attention per head in {best}, one "
+                     f"thread ({elapsed[best]:.1f} s)"
+                     + (f"; the other oracle on the same heads: {others}" if others else ""),
+           "by_oracle": rates}
     if with_dense:
-        out["dense_us_per_step"] = dense_el / done * w.B * w.Hq * 1e6
+        out["dense_us_per_step"] = dense_el[best] / done * w.B * w.Hq * 1e6
     return out
 
 
@@ -957,6 +970,18 @@ def main():
             "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "us_per_step": e2e_step_ms * 1e3}}
+    if rank == 0 and world == 1:
+        try:  # the same step without the flush: L2 as the previous step left it
+            wn = min(args.steps, 200)
+            for _ in range(3):
+                step.timed(flush=False)
+            warm_ms = sum(step.timed(flush=False)[0] for _ in range(wn)) / wn
+            line["warm"] = {"us_per_step": warm_ms * 1e3, "steps": wn,
+                            "gbs": step_bytes(w) / (warm_ms * 1e-3) / 1e9,
+                            "l2": f"not flushed between steps (the step reads "
+                                  f"{step_bytes(w) / 1e6:.0f} MB; L2 holds 126 MB)"}
+        except Exception as e:  # noqa: BLE001  (the flushed figures stand without it)
+            line["warm"] = {"error": repr(e)[:200]}
     step.release()
     if args.mode == "step":
         # the same step as separate calls: per-kernel stage times
