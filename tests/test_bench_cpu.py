@@ -74,3 +74,21 @@ def test_cpu_baseline_head_cap():
     r = bench.time_oracle(dsgen.workload("sweep-B32-H32-T32K-r8-k512"), 30.0, max_heads=2)
     assert r["sample"].startswith("2 head-steps") and r["value"] > 0
     assert r["us_per_step"] > 0 and r["cores"] == 1
+
+
+def test_committed_profiles_are_consistent():
+    """The committed summaries parse, name the commands that made them, and agree with
+    the algorithmic bytes bench.py reports for the same kernel and workload."""
+    prof = os.path.join(ROOT, "profiles")
+    w = dsgen.workload(bench.HEADLINE)
+    ks = open(os.path.join(prof, f"k_step_{w.name}.txt")).read()
+    assert "ncu --set full --clock-control none" in ks
+    kv = dict(l.split(":", 1) for l in ks.splitlines() if ":" in l and not l.startswith("#"))
+    alg = int(kv["algorithmic_bytes_per_launch"].split()[0])
+    assert alg == bench.stage_bytes(w)["decode_step"]
+    total = float(kv["dram_bytes_total"])
+    assert 0.9 < total / alg < 1.2  # no large re-reads
+    tr = open(os.path.join(prof, f"traffic_{w.name}.txt")).read()
+    assert f"dram_bytes_per_launch[k_step]: {total:.0f}" in tr
+    ls = open(os.path.join(prof, f"launches_{w.name}.txt")).read()
+    assert "--clock-control none" in ls and "ds::k_step" in ls
