@@ -22,7 +22,6 @@ each with its own seeded batch): the decode step has no cross-GPU exchange.
 from __future__ import annotations
 
 import argparse
-import ctypes
 import datetime
 import hashlib
 import json

@@ -6,7 +6,6 @@ least one pin must fail.  This is the evidence that the pins constrain every
 step of the oracle, not just that the oracle agrees with itself.
 """
 import importlib.util
-import os
 import types
 
 import pytest
