@@ -181,17 +181,22 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
  *   l_i = scale * (q[b,h,:] . K[b,g(h),i,:]);  w = softmax(l);
  *   O[b,h,:] = sum_i w_i V[b,g(h),i,:];  lse[b,h] = log sum_i exp(l_i).
  * Self-attention computed with the important tokens only (Double Sparsity
- * page, Abstract; Key points 2).  The k rows are split into chunks processed
- * in parallel; each chunk keeps a running max and sum and the chunks are
- * combined by log-sum-exp weights.  fp32 accumulation.
+ * page, Abstract; Key points 2).  The k rows of all heads, head after head,
+ * are cut into equal contiguous ranges, one per warp of a grid of one
+ * 16-warp CTA per SM; each range keeps a running max and sum per head it
+ * touches, and a head shared by several ranges is combined by log-sum-exp
+ * weights (first within a CTA, then across CTAs).  fp32 accumulation.
  *
  * Q: [B,Hq,d] bf16; K, V: [B,Hkv,T_cap,d] bf16; idx: [B*Hq,k] int32 with
  * entries in [0, T) (out-of-range entries are clamped and flagged);
  * O: [B,Hq,d] fp32; lse: [B,Hq] fp32 or NULL.  Requires 1 <= k <= T <= T_cap.
  * ws: ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k) bytes of device
- * memory, zero-filled before its first use (it holds per-head counters that
- * every call leaves at zero again); may be NULL when that size is 0.  Calls
- * that may overlap on the GPU need separate workspaces.
+ * memory, zero-filled before its first use; may be NULL when that size is 0.
+ * Its first 256 KiB hold one arrival counter per head at a fixed place, which
+ * every call leaves at zero again, and the per-range partials follow; so one
+ * buffer of the largest size needed serves any number of calls, of any sizes,
+ * that do not overlap on the GPU.  Calls that may overlap on the GPU need
+ * separate workspaces.
  */
 ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
                            float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
@@ -278,17 +283,25 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
  * cudaFree or other allocating routine.
  *
  * Arguments as for ds_sparse_decode, without ws / ws_bytes.  Returns
- * DS_ERR_WORKSPACE, launching nothing, when the partials these sizes need
- * (ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k)) exceed
- * DS_NOALLOC_SCRATCH_BYTES.
+ * DS_ERR_WORKSPACE, launching nothing, when the workspace these sizes need
+ * (ds_workspace_size(DS_OP_SPARSE_DECODE, dims, T, k)) exceeds
+ * DS_NOALLOC_SCRATCH_BYTES.  With the work plan of ds_sparse_decode that does
+ * not happen for sizes the library accepts: heads are shared by several warps
+ * only when there are fewer heads than warps in the grid (148 CTAs of 16), so
+ * at most 148 + 2367 partials of 528 bytes follow the 256 KiB of counters
+ * (1.6 MB).  Sizes beyond the library's limits (B*Hq > 65535) return
+ * DS_ERR_UNSUPPORTED.
  *
  * The first call on each device looks up the array's device address with
  * that device current (cudaGetSymbolAddress); make that first call outside
- * any stream capture.  All calls on a device share the one array and it keeps
- * the previous call's contents; each call first clears (on `stream`) the
- * per-head counters that must start at zero.  Calls that may overlap on the
- * GPU -- on different streams without an ordering between them -- race on the
- * array and must not be issued.
+ * any stream capture: until the address is known, a call on a stream that is
+ * being captured returns DS_ERR_UNSUPPORTED and launches nothing.  All calls
+ * on a device share the one array and it keeps the previous call's contents.
+ * Its layout is that of the ds_sparse_decode workspace: the per-head counters
+ * sit at its start, are zero when the library is loaded and are left at zero
+ * by every call, so no call has to clear anything first.  Calls that may
+ * overlap on the GPU -- on different streams without an ordering between them
+ * -- race on the array and must not be issued.
  */
 #define DS_NOALLOC_SCRATCH_BYTES (4u << 20)
 ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,

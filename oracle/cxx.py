@@ -67,11 +67,14 @@ def _load():
                                      vp, vp],
                 "dso_hier_topk_f64": [vp, i64, i32, i32, vp],
                 "dso_hier_topk_f32": [vp, i64, i32, i32, vp],
+                "dso_step_heads_mt": [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f64, i32,
+                                      i32, vp, vp, vp, vp],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
-                fn.restype = ctypes.c_int if name == "dso_block_tokens" else None
+                fn.restype = (ctypes.c_int if name in ("dso_block_tokens", "dso_step_heads_mt")
+                              else None)
             _lib = lib
     return _lib
 
@@ -343,3 +346,27 @@ def hier_topk(s, k: int):
 
 def hier_topk_head(s, k: int):
     return hier_topk(np.asarray(s)[None], k)[0]
+
+
+# ---- the per-head step over host threads (CPU baseline) ---------------------------
+
+def step_heads_mt(Qs, Cs, Ls, Ks, Vs, k: int, scale, sparse: bool = True,
+                  dense: bool = False, nthreads: int = 0):
+    """Per head i (query Qs[i] [d], channels Cs[i] [r], label rows Ls[i] [T, r], its
+    KV head's rows Ks[i], Vs[i] [T, d]): the sparse step (score, float32 rounding,
+    top-k, attention) and/or dense attention, the heads spread over nthreads host
+    threads (0: every core).  Returns (O, lse, Od, lsed, threads used)."""
+    Qs, Ks, Vs = (_c(a, np.uint16) for a in (Qs, Ks, Vs))
+    Cs = _c(Cs, np.int32)
+    n, T, d = Ks.shape
+    r = Cs.shape[1]
+    Ls = _c(Ls, np.uint16) if sparse else np.zeros((n, 1, r), np.uint16)
+    O = np.empty((n, d), np.float64)
+    lse = np.empty(n, np.float64)
+    Od = np.empty((n, d), np.float64)
+    lsed = np.empty(n, np.float64)
+    mode = (1 if sparse else 0) | (2 if dense else 0)
+    used = _load().dso_step_heads_mt(_p(Qs), _p(Cs), _p(Ls), _p(Ks), _p(Vs), n, T, d, r, int(k),
+                                     float(scale), mode, int(nthreads), _p(O), _p(lse), _p(Od),
+                                     _p(lsed))
+    return O, lse, Od, lsed, int(used)

@@ -46,10 +46,12 @@
 // double precision (std::exp, std::log); the order of the top-k is decided by
 // std::sort on the stated total order.  Plain loops, no blocking or fusion.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <numeric>
+#include <thread>
 #include <vector>
 
 namespace {
@@ -378,6 +380,58 @@ void dso_hier_topk_f64(const double* s, int64_t rows, int T, int k, int32_t* idx
 }
 void dso_hier_topk_f32(const float* s, int64_t rows, int T, int k, int32_t* idx) {
   for (int64_t i = 0; i < rows; ++i) hier_row(s + i * T, T, k, idx + i * k);
+}
+
+// The decode step of n independent heads spread over host threads (the CPU
+// baseline: the same per-head steps, the heads shared out by a counter).  Head
+// i has the query Qs[i] [d], channel ids Cs[i] [r], label rows Ls[i] [T, r] and
+// its KV head's rows Ks[i], Vs[i] [T, d].  mode bit 1: O2 score in float64,
+// rounded to float32, O3 top-k of k tokens, O4 attention over them -> O[i],
+// lse[i]; mode bit 2: O5 dense attention over all T rows -> Od[i], lsed[i].
+// nthreads <= 0 uses std::thread::hardware_concurrency().  Returns the number
+// of threads used.
+int dso_step_heads_mt(const uint16_t* Qs, const int32_t* Cs, const uint16_t* Ls,
+                      const uint16_t* Ks, const uint16_t* Vs, int n, int T, int d, int r, int k,
+                      double scale, int mode, int nthreads, double* O, double* lse, double* Od,
+                      double* lsed) {
+  if (nthreads <= 0) nthreads = static_cast<int>(std::thread::hardware_concurrency());
+  if (nthreads <= 0) nthreads = 1;
+  std::atomic<int> next{0};
+  auto worker = [&]() {
+    std::vector<double> s(T);
+    std::vector<float> s32(T);
+    std::vector<int32_t> idx(k), all;
+    if (mode & 2) {
+      all.resize(T);
+      std::iota(all.begin(), all.end(), 0);
+    }
+    for (int i = next.fetch_add(1); i < n; i = next.fetch_add(1)) {
+      const uint16_t* q = Qs + static_cast<int64_t>(i) * d;
+      const int32_t* C = Cs + static_cast<int64_t>(i) * r;
+      const uint16_t* K = Ks + static_cast<int64_t>(i) * T * d;
+      const uint16_t* V = Vs + static_cast<int64_t>(i) * T * d;
+      if (mode & 1) {
+        const uint16_t* lab = Ls + static_cast<int64_t>(i) * T * r;
+        for (int t = 0; t < T; ++t) {
+          double acc = 0.0;
+          for (int j = 0; j < r; ++j)
+            acc += bf16_value(q[C[j]]) * bf16_value(lab[static_cast<int64_t>(t) * r + j]);
+          s[t] = acc;
+          s32[t] = static_cast<float>(acc);
+        }
+        topk_row(s32.data(), T, k, idx.data());
+        attend_row(q, K, V, idx.data(), k, d, scale, O + static_cast<int64_t>(i) * d, lse + i,
+                   nullptr);
+      }
+      if (mode & 2)
+        attend_row(q, K, V, all.data(), T, d, scale, Od + static_cast<int64_t>(i) * d, lsed + i,
+                   nullptr);
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nthreads; ++t) pool.emplace_back(worker);
+  for (auto& th : pool) th.join();
+  return nthreads;
 }
 
 }  // extern "C"

@@ -64,8 +64,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed building libds.so")
     if verbose:
         sys.stderr.write(res.stderr)
-    with open(os.path.join(PKG, "ptxas_report.txt"), "w") as fh:
-        fh.write(" ".join(cmd) + "\n" + res.stderr)
+    # register and shared-memory report of the build (a build output, not source)
+    os.makedirs(os.path.join(ROOT, "build"), exist_ok=True)
+    with open(os.path.join(ROOT, "build", "ptxas_report.txt"), "w") as fh:
+        fh.write(res.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -11,6 +11,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ds.h"
 
 #include "attend.cuh"
@@ -26,6 +28,14 @@ namespace {
 using namespace ds;
 
 std::atomic<uint64_t> g_launches{0};
+
+// One NVTX range per C-ABI call (visible in Nsight timelines; a no-op when no
+// tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define DS_TRACE(name) NvtxRange ds_nvtx_range_(name)
 thread_local char g_cuda_err[256] = "no error";
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -89,57 +99,23 @@ ds_status check_dims(const ds_dims& d) {
   return DS_OK;
 }
 
-// ---- split plan for the attention kernels (device independent) -------------
-// Heads are cut into S splits of rows_per_split rows.  S is the smallest count
-// (splits of at least kMinRowsPerSplit rows; sparse splits keep their index
-// list in shared memory, so at most kMaxRowsPerSplitSparse rows) whose grid
-// fills its last wave of kWaveCtas CTAs (148 SMs x 6 resident CTAs) to within
-// 10%, else the one that fills it best.
-constexpr int kWaveCtas = 148 * 6;
-constexpr int kMinRowsPerSplit = 64;
-
-struct SplitPlan {
-  int S;
-  int rows_per_split;
-};
-
-SplitPlan plan_splits(int heads, int rows, bool sparse) {
-  const int s_min = sparse ? (rows + kMaxRowsPerSplitSparse - 1) / kMaxRowsPerSplitSparse : 1;
-  const int s_max = std::max(s_min, std::min(256, rows / kMinRowsPerSplit));
-  int best = s_min;
-  double best_waste = 1e30;
-  for (int S = s_min; S <= s_max; ++S) {
-    const double n = (double)heads * S;
-    const double waves = std::ceil(n / kWaveCtas);
-    const double waste = waves * kWaveCtas / n;  // >= 1; 1 = the last wave is full
-    if (waste < best_waste - 1e-9) {
-      best_waste = waste;
-      best = S;
-    }
-    if (waste <= 1.10) break;
-  }
-  int rps = (rows + best - 1) / best;
-  rps = (rps + 3) & ~3;
-  return {(rows + rps - 1) / rps, rps};
-}
-
-// Workspace: the split partials, then one arrival counter per head.
-size_t partial_bytes(int heads, const SplitPlan& sp) {
-  if (sp.S <= 1) return 0;
-  size_t b = (size_t)heads * sp.S * kPartialStride * sizeof(float) + (size_t)heads * 4;
-  return (b + 255) & ~size_t(255);
-}
-
-size_t attend_smem(const SplitPlan& sp, bool sparse) {
-  size_t b = (size_t)kAttnWarps * kAttnStages * kAttnStageU4 * 16 + kAttnWarps * 132 * 4;
-  if (sparse) b += (size_t)sp.rows_per_split * 4;
-  return b;
-}
+// ---- attention work plan (device independent) -------------------------------
+// attn_plan (attend.cuh): every warp of one wave takes an equal, contiguous
+// range of the heads' rows; the workspace holds the arrival counters at a
+// fixed place, then the partials of the heads that several warps share.
+size_t attend_ws_bytes(int heads, int rows) { return attn_workspace_bytes(attn_plan(heads, rows)); }
 
 // ---- per-device one-time kernel attributes ----------------------------------
 constexpr int kMaxDevices = 64;
 std::once_flag g_attr_once[kMaxDevices];
 cudaError_t g_attr_err[kMaxDevices];
+int g_sm_count[kMaxDevices];
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+}
 
 template <class Kern>
 cudaError_t allow_smem(Kern k, size_t bytes) {
@@ -163,10 +139,8 @@ ds_status ensure_attrs() {
     auto acc = [&r](cudaError_t x) {
       if (r == cudaSuccess) r = x;
     };
-    const size_t attn_max = (size_t)kAttnWarps * kAttnStages * kAttnStageU4 * 16 +
-                            kAttnWarps * 132 * 4 + (size_t)kMaxRowsPerSplitSparse * 4;
-    acc(allow_smem(k_attend<true>, attn_max));
-    acc(allow_smem(k_attend<false>, attn_max));
+    acc(allow_smem(k_attend<true>, kAttnSmemBytes));
+    acc(allow_smem(k_attend<false>, kAttnSmemBytes));
     acc(topk_attrs<ScoresSource>());
     acc(topk_attrs<LabelSource<8>>());
     acc(topk_attrs<LabelSource<16>>());
@@ -185,6 +159,9 @@ ds_status ensure_attrs() {
     acc(allow_smem(k_step<32>, step_max));
     acc(allow_smem(k_step<64>, step_max));
     acc(allow_smem(k_step<128>, step_max));
+    int sms = 0;
+    acc(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    g_sm_count[dev] = sms > 0 ? sms : 148;
     g_attr_err[dev] = r;
   });
   return g_attr_err[dev] == cudaSuccess ? DS_OK : cuda_fail(g_attr_err[dev]);
@@ -283,14 +260,10 @@ ds_status fused_topk(const uint16_t* Q, const int32_t* C, const uint16_t* label,
   return launch_topk(src, idx, d.B * d.Hq, T, k, st);
 }
 
-// Host-side checks of the split plan and workspace (no CUDA calls).
-ds_status check_attend_ws(const ds_dims& d, int rows, bool sparse, const void* ws,
-                          size_t ws_bytes) {
-  const int BH = d.B * d.Hq;
-  const SplitPlan sp = plan_splits(BH, rows, sparse);
-  const size_t need = partial_bytes(BH, sp);
+// Host-side check of the workspace (no CUDA calls).
+ds_status check_attend_ws(const ds_dims& d, int rows, const void* ws, size_t ws_bytes) {
+  const size_t need = attend_ws_bytes(d.B * d.Hq, rows);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return DS_ERR_WORKSPACE;
-  if (sp.S > 65535) return DS_ERR_UNSUPPORTED;
   return DS_OK;
 }
 
@@ -299,8 +272,8 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
                         void* ws, cudaStream_t st, bool idx_per_group = false,
                         int block = 0) {
   const bool sparse = idx != nullptr;
-  const int BH = d.B * d.Hq;
-  const SplitPlan sp = plan_splits(BH, rows, sparse);
+  const int heads = d.B * d.Hq;
+  const AttnPlan pl = attn_plan(heads, rows);
 
   AttnParams p;
   p.Q = static_cast<const uint16_t*>(Q);
@@ -311,24 +284,24 @@ ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const vo
   p.block = block;
   p.O = O;
   p.lse = lse;
-  p.partial = static_cast<float*>(ws);
-  p.arrivals = ws ? reinterpret_cast<uint32_t*>(static_cast<float*>(ws) +
-                                                (size_t)BH * sp.S * kPartialStride)
-                  : nullptr;
+  p.arrivals = pl.slots ? static_cast<uint32_t*>(ws) : nullptr;
+  p.partial = pl.slots ? reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes)
+                       : nullptr;
+  p.heads = heads;
   p.Hq = d.Hq;
   p.Hkv = d.Hkv;
   p.T_cap = d.T_cap;
   p.T = T;
   p.rows = rows;
-  p.rows_per_split = sp.rows_per_split;
+  p.per = pl.per;
+  p.units = pl.units;
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  dim3 grid(d.Hq / d.Hkv, sp.S, d.B * d.Hkv);
-  const size_t smem = attend_smem(sp, sparse);
+  const int grid = (pl.units + kAttnWarps - 1) / kAttnWarps;
   if (sparse)
-    k_attend<true><<<grid, kAttnThreads, smem, st>>>(p);
+    k_attend<true><<<grid, kAttnThreads, kAttnSmemBytes, st>>>(p);
   else
-    k_attend<false><<<grid, kAttnThreads, smem, st>>>(p);
+    k_attend<false><<<grid, kAttnThreads, kAttnSmemBytes, st>>>(p);
   return launched();
 }
 
@@ -367,7 +340,7 @@ bool step_fused(const ds_dims& d, int T, int k, int* chunk_out, size_t* smem_out
 // scores.  Returns the total; *scores_off gets the offset of the scores (0: none).
 size_t step_fallback_ws(const ds_dims& d, int T, int k, size_t* scores_off) {
   const int BH = d.B * d.Hq;
-  size_t n = partial_bytes(BH, plan_splits(BH, k, true));
+  size_t n = attend_ws_bytes(BH, k);
   size_t off = 0;
   if (prefer_score_then_select(d.r, T)) {
     off = (n + 255) & ~(size_t)255;
@@ -408,9 +381,9 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
   switch (op) {
     case DS_OP_SPARSE_DECODE:
       if (k < 1 || k > T) return 0;
-      return partial_bytes(BH, plan_splits(BH, k, true));
+      return attend_ws_bytes(BH, k);
     case DS_OP_DECODE:
-      return partial_bytes(BH, plan_splits(BH, T, false));
+      return attend_ws_bytes(BH, T);
     case DS_OP_DECODE_STEP: {
       if (k < 1 || k > T) return 0;
       int chunk;
@@ -420,10 +393,10 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
     }
     case DS_OP_BLOCK_SPARSE_DECODE:  // k: kept rows, blocks x block size
       if (k < 1) return 0;
-      return partial_bytes(BH, plan_splits(BH, k, true));
-    case DS_OP_GROUP_SPARSE_DECODE:  // the same split plan as the per-head call
+      return attend_ws_bytes(BH, k);
+    case DS_OP_GROUP_SPARSE_DECODE:  // the same plan as the per-head call
       if (k < 1 || k > T) return 0;
-      return partial_bytes(BH, plan_splits(BH, k, true));
+      return attend_ws_bytes(BH, k);
     case DS_OP_CALIBRATE: {
       if (k < 1) return 0;  // k: calibration queries per head
       const size_t nck = (T + kAbsumRows - 1) / kAbsumRows, ncq = (k + kAbsumRows - 1) / kAbsumRows;
@@ -436,6 +409,7 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
 }
 
 ds_status ds_device_status(uint32_t* bits, int32_t clear, ds_stream_t stream) {
+  DS_TRACE("ds_device_status");
   if (!bits) return DS_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -453,6 +427,7 @@ ds_status ds_device_status(uint32_t* bits, int32_t clear, ds_stream_t stream) {
 
 ds_status ds_label_append(const void* K, const int32_t* C, void* label, ds_dims dims, int32_t t0,
                           int32_t n, ds_stream_t stream) {
+  DS_TRACE("ds_label_append");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!K || !C || !label || !aligned16(K) || !aligned16(C) || !aligned16(label))
@@ -472,6 +447,7 @@ ds_status ds_label_append(const void* K, const int32_t* C, void* label, ds_dims 
 
 ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* scores,
                    ds_dims dims, int32_t T, ds_stream_t stream) {
+  DS_TRACE("ds_score");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !C || !label || !scores || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
@@ -484,6 +460,7 @@ ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* sc
 
 ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int32_t k, void* ws,
                   size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_topk");
   (void)ws;
   (void)ws_bytes;
   if (!scores || !idx || !aligned16(scores) || !aligned16(idx)) return DS_ERR_INVALID_ARG;
@@ -496,6 +473,7 @@ ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int3
 
 ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
                         int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream) {
+  DS_TRACE("ds_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !C || !label || !idx || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
@@ -531,13 +509,14 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
 ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const int32_t* idx,
                            float* O, float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
                            void* ws, size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_sparse_decode");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
       !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
-  s = check_attend_ws(dims, k, true, ws, ws_bytes);
+  s = check_attend_ws(dims, k, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
@@ -549,13 +528,14 @@ ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const in
 ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float* lse,
                     ds_dims dims, int32_t T, float scale, void* ws, size_t ws_bytes,
                     ds_stream_t stream) {
+  DS_TRACE("ds_decode");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
       !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
-  s = check_attend_ws(dims, T, false, ws, ws_bytes);
+  s = check_attend_ws(dims, T, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
@@ -567,29 +547,44 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
 }  // extern "C"
 
 // ---- sparse decode with library-owned scratch ---------------------------------
-// For callers that must not allocate device memory: the split partials live in
-// this fixed file-scope array instead of a caller workspace.  Every call on a
-// device shares it, so calls that overlap on the GPU race on it.
+// For callers that must not allocate device memory: the workspace of
+// ds_sparse_decode -- arrival counters at its start, then the split partials --
+// lives in this fixed file-scope array instead.  It is zero when the library is
+// loaded and every call leaves its counters at zero, so no call has to clear
+// anything first.  Every call on a device shares it, so calls that overlap on
+// the GPU race on it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DS_NOALLOC_SCRATCH_BYTES];
+static_assert(kCounterBytes < DS_NOALLOC_SCRATCH_BYTES, "the counters fit the scratch array");
 
 namespace {
 std::once_flag g_scratch_once[kMaxDevices];
-void* g_scratch_addr[kMaxDevices];
+std::atomic<void*> g_scratch_addr[kMaxDevices];
 cudaError_t g_scratch_err[kMaxDevices];
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name is only a host-side handle, so the address is looked up once
-// per device, with that device current.
-ds_status noalloc_scratch(void** out) {
+// per device, with that device current.  The lookup is refused while `stream`
+// is being captured into a graph (the first call must come before capture).
+ds_status noalloc_scratch(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return DS_ERR_UNSUPPORTED;
-  std::call_once(g_scratch_once[dev], [dev] {
-    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_noalloc_scratch);
-  });
-  if (g_scratch_err[dev] != cudaSuccess) return cuda_fail(g_scratch_err[dev]);
-  *out = g_scratch_addr[dev];
+  void* a = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (a == nullptr) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (cap != cudaStreamCaptureStatusNone) return DS_ERR_UNSUPPORTED;
+    std::call_once(g_scratch_once[dev], [dev] {
+      void* p = nullptr;
+      g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (g_scratch_err[dev] == cudaSuccess) g_scratch_addr[dev].store(p, std::memory_order_release);
+    });
+    if (g_scratch_err[dev] != cudaSuccess) return cuda_fail(g_scratch_err[dev]);
+    a = g_scratch_addr[dev].load(std::memory_order_acquire);
+  }
+  *out = a;
   return DS_OK;
 }
 }  // namespace
@@ -598,30 +593,23 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
                                               const int32_t* idx, float* O, float* lse,
                                               ds_dims dims, int32_t T, int32_t k, float scale,
                                               ds_stream_t stream) {
+  DS_TRACE("ds_sparse_decode_noalloc");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
       !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
-  const int BH = dims.B * dims.Hq;
-  const SplitPlan sp = plan_splits(BH, k, true);
-  const size_t need = partial_bytes(BH, sp);
+  const size_t need = attend_ws_bytes(dims.B * dims.Hq, k);
   if (need > DS_NOALLOC_SCRATCH_BYTES) return DS_ERR_WORKSPACE;
-  if (sp.S > 65535) return DS_ERR_UNSUPPORTED;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
   void* scratch = nullptr;
   if (need > 0) {
-    s = noalloc_scratch(&scratch);
+    s = noalloc_scratch(stream, &scratch);
     if (s != DS_OK) return s;
-    // the arrival counters after the partials must start at zero
-    const size_t counters = (size_t)BH * sp.S * kPartialStride * sizeof(float);
-    cudaError_t e = cudaMemsetAsync(static_cast<char*>(scratch) + counters, 0,
-                                    (size_t)BH * sizeof(uint32_t), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
   }
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
 }
@@ -651,7 +639,7 @@ ds_status decode_step(const void* Q, const void* K_new, const void* V_new, const
   const bool fused = step_fused(dims, T, k, &chunk, &smem);
   size_t scores_off = 0;
   if (!fused) {
-    s = check_attend_ws(dims, k, true, ws, ws_bytes);
+    s = check_attend_ws(dims, k, ws, ws_bytes);
     if (s != DS_OK) return s;
     if (ws_bytes < step_fallback_ws(dims, T, k, &scores_off)) return DS_ERR_WORKSPACE;
     const bool vec = dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 ||
@@ -718,6 +706,7 @@ extern "C" ds_status ds_decode_step(const void* Q, const void* K, const void* V,
                                     ds_dims dims, int32_t T, int32_t k, float scale,
                                     int32_t append, void* ws, size_t ws_bytes,
                                     ds_stream_t stream) {
+  DS_TRACE("ds_decode_step");
   return decode_step(Q, nullptr, nullptr, K, V, C, label, idx, O, lse, dims, T, k, scale, append,
                      ws, ws_bytes, stream);
 }
@@ -727,6 +716,7 @@ extern "C" ds_status ds_decode_step_kv(const void* Q, const void* K_new, const v
                                        int32_t* idx, float* O, float* lse, ds_dims dims,
                                        int32_t T, int32_t k, float scale, void* ws,
                                        size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_decode_step_kv");
   if (!K_new || !V_new) return DS_ERR_INVALID_ARG;
   return decode_step(Q, K_new, V_new, K, V, C, label, idx, O, lse, dims, T, k, scale, 1, ws,
                      ws_bytes, stream);
@@ -735,6 +725,7 @@ extern "C" ds_status ds_decode_step_kv(const void* Q, const void* K_new, const v
 extern "C" ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_dims dims,
                                   int32_t T, int32_t* C, float* importance, void* ws,
                                   size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_calibrate");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Qc || !K || !C || !aligned16(Qc) || !aligned16(K) || !aligned16(C))
@@ -779,6 +770,7 @@ ds_status launch_group_score(const uint16_t* Q, const int32_t* C, const uint16_t
 extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
                                          float* group_scores, int32_t* idx, ds_dims dims,
                                          int32_t T, int32_t k, ds_stream_t stream) {
+  DS_TRACE("ds_group_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !C || !label || !group_scores || !idx || !aligned16(Q) || !aligned16(C) ||
@@ -810,13 +802,14 @@ extern "C" ds_status ds_group_sparse_decode(const void* Q, const void* K, const 
                                             const int32_t* idx, float* O, float* lse,
                                             ds_dims dims, int32_t T, int32_t k, float scale,
                                             void* ws, size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_group_sparse_decode");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
       !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
-  s = check_attend_ws(dims, k, true, ws, ws_bytes);
+  s = check_attend_ws(dims, k, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
@@ -843,6 +836,7 @@ ds_status launch_block_score(const uint16_t* Q, const int32_t* C, const uint16_t
 extern "C" ds_status ds_block_score_topk(const void* Q, const int32_t* C, const void* label,
                                          float* block_scores, int32_t* bidx, ds_dims dims,
                                          int32_t T, int32_t bs, int32_t kb, ds_stream_t stream) {
+  DS_TRACE("ds_block_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !C || !label || !block_scores || !bidx || !aligned16(Q) || !aligned16(C) ||
@@ -874,6 +868,7 @@ extern "C" ds_status ds_block_sparse_decode(const void* Q, const void* K, const 
                                             ds_dims dims, int32_t T, int32_t bs, int32_t kb,
                                             float scale, void* ws, size_t ws_bytes,
                                             ds_stream_t stream) {
+  DS_TRACE("ds_block_sparse_decode");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !K || !V || !bidx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
@@ -883,7 +878,7 @@ extern "C" ds_status ds_block_sparse_decode(const void* Q, const void* K, const 
   if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
   if (kb < 1 || kb > (T + bs - 1) / bs) return DS_ERR_INVALID_ARG;
   const int rows = kb * bs;
-  s = check_attend_ws(dims, rows, true, ws, ws_bytes);
+  s = check_attend_ws(dims, rows, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
@@ -908,6 +903,7 @@ ds_status launch_hier(const uint16_t* Q, const int32_t* C, const uint16_t* label
 extern "C" ds_status ds_hier_score_topk(const void* Q, const int32_t* C, const void* label,
                                         int32_t* idx, ds_dims dims, int32_t T, int32_t k,
                                         ds_stream_t stream) {
+  DS_TRACE("ds_hier_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!Q || !C || !label || !idx || !aligned16(Q) || !aligned16(C) || !aligned16(label) ||
@@ -932,6 +928,7 @@ extern "C" ds_status ds_hier_score_topk(const void* Q, const int32_t* C, const v
 
 extern "C" ds_status ds_kv_append(const void* K_new, const void* V_new, void* K, void* V,
                                   ds_dims dims, int32_t t, ds_stream_t stream) {
+  DS_TRACE("ds_kv_append");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
   if (!K_new || !V_new || !K || !V || !aligned16(K_new) || !aligned16(V_new) || !aligned16(K) ||

@@ -127,23 +127,19 @@ def test_workspace_checked_before_launch():
 
 def test_workspace_sizes():
     lib = ds.lib()
-    # short rows: no split, no workspace
+    # short rows: every warp takes whole heads, nothing to merge, no workspace
     d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
-    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 100) == 0
+    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 16) == 0
     assert lib.ds_workspace_size(ds.OP_TOPK, d, 32768, 512) == 0
     assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == 0
-    # heads that fill whole waves of the grid on their own (148 SMs x 6): no split
-    d = _dims(B=8, Hq=111, Hkv=111, T_cap=32768, r=8)
-    assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 2048) == 0
-    # otherwise the split count fills the last wave: partials + one counter per head
-    d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
+    # heads shared by warps: 256 KiB of counters, then 132 floats per slot
     n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 2048)
-    S = round((n - 1024 * 4) / (1024 * 132 * 4))
-    assert S >= 2 and n >= 1024 * (S * 132 * 4 + 4) and n % 256 == 0
-    # long single sequence: split, 132 floats per split, 256-byte rounded
+    assert n > 256 * 1024 and n % 256 == 0
+    assert (n - 256 * 1024) // (132 * 4) >= 1024
+    # long single sequence
     d = _dims(B=1, Hq=32, Hkv=32, T_cap=262144, r=8)
     n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 262144, 16384)
-    assert n > 0 and n % 256 == 0 and (n // (32 * 132 * 4)) >= 2
+    assert n > 256 * 1024 and n % 256 == 0
     # invalid sizes give 0
     assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 0, 1) == 0
     assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 100, 101) == 0
@@ -297,35 +293,40 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     assert "libds.so is missing" in res.stderr
 
 
-def _plan(heads, rows, sparse):
-    """The documented split rule: at most 2048 rows per sparse split, at least 64
-    rows, the smallest split count whose grid fills its last wave of 148 x 6 CTAs
-    to within 10% (else the best filled), rows per split a multiple of 4."""
-    import math
-    wave = 148 * 6
-    s_min = -(-rows // 2048) if sparse else 1
-    s_max = max(s_min, min(256, rows // 64))
-    best, best_waste = s_min, math.inf
-    for S in range(s_min, s_max + 1):
-        n = heads * S
-        waste = math.ceil(n / wave) * wave / n
-        if waste < best_waste - 1e-9:
-            best, best_waste = S, waste
-        if waste <= 1.10:
-            break
-    rps = -(-rows // best)
-    rps = (rps + 3) & ~3
-    return -(-rows // rps)
+def _plan(heads, rows):
+    """The documented work plan: a grid of 148 CTAs of 16 warps; the R = heads *
+    rows rows are cut into ranges of `per` rows, per = ceil(R / (148 * 16)) but
+    at least 16, rounded up to a multiple of 4.  When per >= rows every range is
+    a whole number of heads and no workspace is needed; otherwise CTA c and head
+    h share partial slot c + h."""
+    R = heads * rows
+    per = max(-(-R // (148 * 16)), 16)
+    per = (per + 3) & ~3
+    if per >= rows:
+        return 0
+    units = -(-R // per)
+    return -(-units // 16) + heads
 
 
 @pytest.mark.parametrize("B,H,T,k", [(1, 32, 262144, 16384), (32, 32, 32768, 512),
                                      (32, 32, 32768, 2048), (8, 32, 4096, 256),
                                      (16, 64, 16384, 1024), (1, 4, 1000, 1000),
-                                     (3, 7, 5000, 300), (1, 1, 300000, 4000)])
-def test_split_plan_follows_the_documented_rule(B, H, T, k):
+                                     (3, 7, 5000, 300), (1, 1, 300000, 4000),
+                                     (32, 32, 32768, 12)])
+def test_work_plan_follows_the_documented_rule(B, H, T, k):
     lib = ds.lib()
     d = _dims(B=B, Hq=H, Hkv=H, T_cap=T, r=8)
-    for op, rows, sparse in ((ds.OP_SPARSE_DECODE, k, True), (ds.OP_DECODE, T, False)):
-        S = _plan(B * H, rows, sparse)
-        want = 0 if S <= 1 else (B * H * S * 132 * 4 + B * H * 4 + 255) // 256 * 256
-        assert lib.ds_workspace_size(op, d, T, k if sparse else T) == want, (op, S)
+    for op, rows in ((ds.OP_SPARSE_DECODE, k), (ds.OP_DECODE, T)):
+        slots = _plan(B * H, rows)
+        want = 0 if slots == 0 else (256 * 1024 + slots * 132 * 4 + 255) // 256 * 256
+        assert lib.ds_workspace_size(op, d, T, k if op == ds.OP_SPARSE_DECODE else T) == want, \
+            (op, slots)
+
+
+def test_binding_noalloc_limit_matches_the_header():
+    """The binding's copy of DS_NOALLOC_SCRATCH_BYTES is the header's value."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "ds.h")).read()
+    m = re.search(r"#define DS_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m, "DS_NOALLOC_SCRATCH_BYTES not found in include/ds.h"
+    assert ds.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

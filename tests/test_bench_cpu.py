@@ -29,8 +29,10 @@ def test_reference_arm_prints_one_contract_line():
     assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0
     assert d["config"]["workload"] == "llama2-7b-B8-H32-T4K"
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"]
-    assert "C++" in cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] == os.cpu_count() and cb["value"] == d["value"]
+    assert "C++" in cb["sample"] and "std::thread" in cb["sample"]
+    # the same configuration as the GPU arm reports
+    assert d["config"]["path"] == "step" and "l2" in d["config"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
@@ -68,10 +70,15 @@ def test_traffic_profile_used_only_for_the_profiled_sources(tmp_path, monkeypatc
     assert bench.profiled_traffic("k_step") is None
 
 
-def test_cpu_baseline_head_cap():
-    r = bench.time_oracle(dsgen.workload("sweep-B32-H32-T32K-r8-k512"), 30.0, max_heads=2)
-    assert r["sample"].startswith("2 head-steps") and r["value"] > 0
-    assert r["us_per_step"] > 0 and r["cores"] == 1
+def test_cpu_baseline_bounded_sample_on_every_core():
+    """A workload too large for the byte budget is timed on a seeded sample of its
+    heads, every host core running the C++ oracle; the dense oracle beside it."""
+    w = dsgen.workload("sweep-B32-H32-T32K-r8-k512")
+    per_head = w.T * w.d * 2 * 2 + w.T * w.r * 2
+    r = bench.time_oracle(w, 0.5, with_dense=True, max_bytes=3 * per_head)
+    assert "over 3 of the 1024 heads" in r["sample"] and r["value"] > 0
+    assert r["us_per_step"] > 0 and r["cores"] == os.cpu_count()
+    assert r["dense_us_per_step"] > 0 and r["dense_gbs"] > 0
 
 
 def test_committed_profiles_are_consistent():

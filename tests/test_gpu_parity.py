@@ -313,12 +313,30 @@ def test_errors_on_device_launch_nothing():
 # the named workloads at full size, sampled heads checked one by one
 
 FULL = ["tiny-B1-H4-T1K", "llama2-7b-B8-H32-T4K", "gqa-B16-Hq64-Hkv8-T16K",
-        "long-B1-H32-T256K", "sweep-B32-H32-T32K-r8-k2048"]
+        "long-B1-H32-T256K"] + [n for n in dsgen.ORDER if n.startswith("sweep")]
+
+# the inputs of the last workload set, kept while the next test uses the same
+# set (the nine sweep cells share one)
+_INPUTS = {}
+
+
+def _inputs(w):
+    key = (w.seed, w.B, w.Hq, w.Hkv, w.T)
+    if key not in _INPUTS:
+        for old in _INPUTS.values():
+            old.free()
+        _INPUTS.clear()
+        _INPUTS[key] = gu.Inputs(w)
+    inp = _INPUTS[key]
+    inp.C = dsgen.channels(w, w.r)
+    inp.dC = gu.dev_i32(inp.C)
+    inp.r = w.r
+    return inp
 
 
 def _full_step(name):
     w = dsgen.workload(name)
-    inp = gu.Inputs(w)
+    inp = _inputs(w)
     BH = w.B * w.Hq
     label = _label_dev(inp, w.T)
     scores = torch.empty((BH, w.T), dtype=torch.float32, device="cuda")
@@ -331,12 +349,27 @@ def _full_step(name):
     Od = torch.empty_like(O)
     lsed = torch.empty_like(lse)
     ds.decode(inp.dQ, inp.dK, inp.dV, Od, w.T, w.scale, lse=lsed)
+    # the decode step in the launch configuration the benchmark times (label row
+    # of the newest token appended, selection, attention)
+    idx_st = torch.empty_like(idx)
+    O_st = torch.empty_like(O)
+    ds.decode_step(inp.dQ, inp.dK, inp.dV, inp.dC, label, idx_st, O_st, w.T, w.scale,
+                   append=True)
     torch.cuda.synchronize()
+    assert torch.equal(idx_st, idx)
+    assert (O_st - O).abs().max().item() <= 1e-5
+    del label
     return w, inp, scores, idx, O, lse, Od, lsed
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_workload_sampled_heads(name):
+    """Every named workload at full size: scores, bit-exact top-k, selection and
+    attention on sampled heads against the numpy oracle, and on four of them
+    against the C++ oracle as well; dense attention on the first cell of each
+    input set."""
+    import oracle.cxx as cxx
+
     w, inp, scores, idx, O, lse, Od, lsed = _full_step(name)
     n_sample = w.B * w.Hq if w.B * w.Hq <= 64 else 12
     heads = gu.sample_heads(w.B, w.Hq, n_sample, seed=1)
@@ -344,7 +377,8 @@ def test_full_workload_sampled_heads(name):
     I = idx.cpu().numpy().reshape(w.B, w.Hq, w.k)
     On, Ln, Odn, Ldn = (t.cpu().numpy() for t in (O, lse, Od, lsed))
     worst = {"sparse": 0.0, "dense": 0.0}
-    for b, h in heads:
+    with_dense = not name.startswith("sweep") or name.endswith("r8-k512")
+    for i, (b, h) in enumerate(heads):
         g = h // w.G
         Kbg, Vbg = inp.K[b, g], inp.V[b, g]
         lab = oracle.label_head(Kbg, inp.C[h])
@@ -368,16 +402,63 @@ def test_full_workload_sampled_heads(name):
         e = np.abs(On[b, h] - o).max()
         worst["sparse"] = max(worst["sparse"], e)
         assert e <= SPARSE_TOL and abs(Ln[b, h] - l) <= 1e-3 * (1 + abs(l))
-        od, ld, _ = oracle.attend_head(inp.Q[b, h], Kbg, Vbg, np.arange(w.T), w.scale)
-        e = np.abs(Odn[b, h] - od).max()
-        worst["dense"] = max(worst["dense"], e)
-        assert e <= DENSE_TOL and abs(Ldn[b, h] - ld) <= 1e-3 * (1 + abs(ld))
+        if with_dense or i < 2:
+            od, ld, _ = oracle.attend_head(inp.Q[b, h], Kbg, Vbg, np.arange(w.T), w.scale)
+            e = np.abs(Odn[b, h] - od).max()
+            worst["dense"] = max(worst["dense"], e)
+            assert e <= DENSE_TOL and abs(Ldn[b, h] - ld) <= 1e-3 * (1 + abs(ld))
+        if i < 4:
+            # the C++ oracle: label bits, its fp32 scores' top-k, selection, O
+            labx = cxx.label_head(Kbg, inp.C[h])
+            assert np.array_equal(labx, lab)
+            sx = cxx.score_head(inp.Q[b, h], inp.C[h], labx)
+            ds.topk(gu.dev_f32(cxx.to_f32(sx)[None]), it)
+            assert np.array_equal(it.cpu().numpy()[0], cxx.topk_head(cxx.to_f32(sx), w.k))
+            sxk = np.sort(sx)[::-1][w.k - 1]
+            assert np.all(sx[sel] >= sxk - 1e-3 * (abs(sxk) + 1))
+            ox, lx, _ = cxx.attend_head(inp.Q[b, h], Kbg, Vbg, sel, w.scale)
+            assert np.abs(On[b, h] - ox).max() <= SPARSE_TOL
+            assert abs(Ln[b, h] - lx) <= 1e-3 * (1 + abs(lx))
     if w.n_hh:
         pos = dsgen.hh_positions(w)
         for h in range(w.Hq):
             assert set(pos[h].tolist()) <= set(I[0, h].tolist())
     print(f"{name}: max abs err sparse {worst['sparse']:.3g} dense {worst['dense']:.3g}")
-    inp.free()
+    if not name.startswith("sweep"):
+        for old in _INPUTS.values():
+            old.free()
+        _INPUTS.clear()
+
+
+def test_full_sweep_every_channel_every_token_equals_dense():
+    """The sweep's r = d, k = T cell at full size (B32 H32 T32K): the whole sparse
+    pipeline with every channel and every token keeps every token and equals
+    dense attention; dense matches the oracle on sampled heads."""
+    base = dsgen.workload("sweep-B32-H32-T32K-r8-k512")
+    w = base.with_(name="sweep-B32-H32-T32K-r128-kT", r=base.d, k=base.T)
+    inp = _inputs(w)  # the sweep's input set (kept from the cells above)
+    BH = w.B * w.Hq
+    label = _label_dev(inp, w.T)
+    idx = torch.empty((BH, w.T), dtype=torch.int32, device="cuda")
+    ds.score_topk(inp.dQ, inp.dC, label, idx, w.T)
+    assert torch.equal(idx, torch.arange(w.T, dtype=torch.int32, device="cuda").expand(BH, -1))
+    idx.fill_(-1)
+    O_s = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    ds.decode_step(inp.dQ, inp.dK, inp.dV, inp.dC, label, idx, O_s, w.T, w.scale, append=True)
+    assert torch.equal(idx, torch.arange(w.T, dtype=torch.int32, device="cuda").expand(BH, -1))
+    del label
+    O_d = torch.empty_like(O_s)
+    ds.decode(inp.dQ, inp.dK, inp.dV, O_d, w.T, w.scale)
+    torch.cuda.synchronize()
+    assert (O_s - O_d).abs().max().item() < 1e-5
+    Odn = O_d.cpu().numpy()
+    for b, h in gu.sample_heads(w.B, w.Hq, 6, seed=3):
+        od, _, _ = oracle.attend_head(inp.Q[b, h], inp.K[b, h], inp.V[b, h], np.arange(w.T),
+                                      w.scale)
+        assert np.abs(Odn[b, h] - od).max() <= DENSE_TOL
+    for old in _INPUTS.values():
+        old.free()
+    _INPUTS.clear()
 
 
 @pytest.mark.parametrize("B,H,T,k", [(1, 2, 5000, 1234), (2, 3, 70000, 20000)])

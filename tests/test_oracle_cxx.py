@@ -161,3 +161,30 @@ def test_cxx_rows_beside_the_path_agree_with_numpy_oracle():
     s32 = cxx.sparse_step(Q, K, V, C, w.k, w.scale)["s32"]
     for k in (1, 5, 24, 300):
         assert np.array_equal(oracle.hier_topk(s32, k), cxx.hier_topk(s32, k))
+
+
+def test_threaded_step_equals_the_per_head_oracle():
+    """The C++ oracle's multi-threaded driver (the CPU baseline) gives, head by
+    head, the numpy oracle's sparse step and dense attention."""
+    import dsgen
+    w = dsgen.Workload("mt", B=2, Hq=6, Hkv=2, T=700, r=8, k=37, n_out=8, seed=321)
+    Q, K, V = dsgen.qkv(w)
+    C = dsgen.channels(w)
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    Qs = np.stack([Q[b, h] for b, h in heads])
+    Ks = np.stack([K[b, h // w.G] for b, h in heads])
+    Vs = np.stack([V[b, h // w.G] for b, h in heads])
+    Cs = np.stack([C[h] for _, h in heads])
+    Ls = np.stack([oracle.label_head(Ks[i], Cs[i]) for i in range(len(heads))])
+    O, L, Od, Ld, used = cxx.step_heads_mt(Qs, Cs, Ls, Ks, Vs, w.k, w.scale, dense=True,
+                                           nthreads=3)
+    assert used == 3
+    for i in range(len(heads)):
+        s = oracle.to_f32(oracle.score_head(Qs[i], Cs[i], Ls[i]))
+        o, l, _ = oracle.attend_head(Qs[i], Ks[i], Vs[i], oracle.topk_head(s, w.k), w.scale)
+        assert np.abs(O[i] - o).max() <= 1e-12 and abs(L[i] - l) <= 1e-12
+        od, ld, _ = oracle.attend_head(Qs[i], Ks[i], Vs[i], np.arange(w.T), w.scale)
+        assert np.abs(Od[i] - od).max() <= 1e-12 and abs(Ld[i] - ld) <= 1e-12
+    # sparse only, all cores
+    O2, L2, _, _, used2 = cxx.step_heads_mt(Qs, Cs, Ls, Ks, Vs, w.k, w.scale)
+    assert used2 >= 1 and np.array_equal(O2, O) and np.array_equal(L2, L)
