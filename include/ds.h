@@ -98,7 +98,10 @@ enum {
 /* Device status bits (ds_device_status). */
 enum {
   DS_DEV_BAD_CHANNEL = 1u, /* a channel id in C was outside [0, d); masked  */
-  DS_DEV_BAD_INDEX = 2u    /* a token index was outside [0, T); clamped     */
+  DS_DEV_BAD_INDEX = 2u,   /* a token index was outside [0, T); clamped     */
+  DS_DEV_TIMEOUT = 4u      /* a bounded in-kernel wait ran out: that call's
+                              results are invalid (the kernel returned
+                              instead of hanging)                           */
 };
 
 /*
@@ -164,15 +167,22 @@ ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int3
 /*
  * ds_score_topk -- ds_score followed by ds_topk.
  *
- * Same results as the two calls (same fp32 scores, same index set).  With
- * scores == NULL: one launch that computes the scores while selecting and
- * never writes them.  With a scores buffer ([B*Hq, T] fp32, written): the same
- * one launch, except for r >= 16 and T > 4096, where the scores are written
- * first and the selection reads them (two launches; faster there).  Limits as
- * for ds_topk.  Needs no workspace.
+ * Same results as the two calls (same fp32 scores, same index set).  With a
+ * workspace of ds_workspace_size(DS_OP_SCORE_TOPK, dims, T, k) bytes (nonzero
+ * when r is 8, 16, 32, 64 or 128 and 4096 < T <= 32768): one launch that
+ * scores tiles of every head, keeps each token's 16-bit key prefix in the
+ * workspace, and selects each head in the CTA that finishes its last tile.
+ * Otherwise (no workspace, or other sizes): with scores == NULL one launch
+ * that computes the scores while selecting; with a scores buffer the same
+ * launch, except for r >= 16 and T > 4096, where the scores are written first
+ * and the selection reads them (two launches).  scores ([B*Hq, T] fp32) is
+ * written when given.  ws: device memory, zero-filled before its first use
+ * (its first 256 KiB hold per-head counters that every call leaves at zero);
+ * may be NULL.  Limits as for ds_topk.
  */
 ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
-                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream);
+                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, void* ws,
+                        size_t ws_bytes, ds_stream_t stream);
 
 /*
  * ds_sparse_decode -- exact softmax attention over the selected tokens.
@@ -217,7 +227,8 @@ ds_status ds_sparse_decode(const void* Q, const void* K, const void* V, const in
  * 32, 64 or 128, k <= 8192, B*Hq <= 296 (one wave of two CTAs per SM) and the
  * head's selection fits one CTA; otherwise the three calls are issued on
  * `stream` (the selection through a score buffer in the workspace when
- * r >= 16 and T > 4096, see ds_score_topk).  idx: [B*Hq, k] int32
+ * r >= 16 and T > 4096, or the one-launch selection, see ds_score_topk).
+ * idx: [B*Hq, k] int32
  * (required).  O and lse as for ds_sparse_decode; the attention's summation
  * order may differ from ds_sparse_decode's (fp32 rounding only).  ws:
  * ds_workspace_size(DS_OP_DECODE_STEP, dims, T, k) bytes, zero-filled before

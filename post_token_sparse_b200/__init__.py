@@ -34,7 +34,7 @@ LIB_PATH = os.path.join(_HERE, "libds.so")
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
 (OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK,
  OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE) = range(10)
-DEV_BAD_CHANNEL, DEV_BAD_INDEX = 1, 2
+DEV_BAD_CHANNEL, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
 
 
 class DsError(RuntimeError):
@@ -66,7 +66,7 @@ def _load():
         "ds_label_append": [vp, vp, vp, Dims, i32, i32, vp],
         "ds_score": [vp, vp, vp, vp, Dims, i32, vp],
         "ds_topk": [vp, vp, i32, i32, i32, vp, ctypes.c_size_t, vp],
-        "ds_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
+        "ds_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp, ctypes.c_size_t, vp],
         "ds_sparse_decode": [vp, vp, vp, vp, vp, vp, Dims, i32, i32, ctypes.c_float, vp,
                              ctypes.c_size_t, vp],
         "ds_decode": [vp, vp, vp, vp, vp, Dims, i32, ctypes.c_float, vp, ctypes.c_size_t, vp],
@@ -203,15 +203,21 @@ def topk(scores, idx):
                         BH, T, k, None, 0, _stream(scores.device)), "ds_topk")
 
 
-def score_topk(Q, C, label, idx, T: int, scores=None):
+def score_topk(Q, C, label, idx, T: int, scores=None, ws=None):
+    """Top-k of the channel-sparse scores; ws: the workspace of OP_SCORE_TOPK (made
+    here when None and the sizes use one)."""
     B, Hq, d = Q.shape
     _, _, T_cap, r = label.shape
     dims = Dims(B, Hq, Hq, d, T_cap, r)
     k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_SCORE_TOPK, dims, T, k, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(_lib.ds_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
                               _ptr(label, torch.bfloat16, "label"),
                               _ptr(scores, torch.float32, "scores"),
-                              _ptr(idx, torch.int32, "idx"), dims, T, k, _stream(Q.device)),
+                              _ptr(idx, torch.int32, "idx"), dims, T, k,
+                              _ptr(ws, None, "ws"), nbytes, _stream(Q.device)),
            "ds_score_topk")
 
 
@@ -355,7 +361,8 @@ def calibrate(Qc, K, C, T: int, importance=None, ws=None):
 
 
 def device_status(clear: bool = True, device=None) -> int:
-    """Status bits kernels set on the current device (DEV_BAD_CHANNEL, DEV_BAD_INDEX)."""
+    """Status bits kernels set on the current device (DEV_BAD_CHANNEL, DEV_BAD_INDEX,
+    DEV_TIMEOUT)."""
     bits = ctypes.c_uint32(0)
     _check(_lib.ds_device_status(ctypes.byref(bits), int(clear), _stream(device)),
            "ds_device_status")

@@ -21,6 +21,7 @@
 #include "label.cuh"
 #include "score.cuh"
 #include "step.cuh"
+#include "select.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -109,13 +110,7 @@ size_t attend_ws_bytes(int heads, int rows) { return attn_workspace_bytes(attn_p
 constexpr int kMaxDevices = 64;
 std::once_flag g_attr_once[kMaxDevices];
 cudaError_t g_attr_err[kMaxDevices];
-int g_sm_count[kMaxDevices];
 
-int sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
-}
 
 template <class Kern>
 cudaError_t allow_smem(Kern k, size_t bytes) {
@@ -159,9 +154,6 @@ ds_status ensure_attrs() {
     acc(allow_smem(k_step<32>, step_max));
     acc(allow_smem(k_step<64>, step_max));
     acc(allow_smem(k_step<128>, step_max));
-    int sms = 0;
-    acc(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    g_sm_count[dev] = sms > 0 ? sms : 148;
     g_attr_err[dev] = r;
   });
   return g_attr_err[dev] == cudaSuccess ? DS_OK : cuda_fail(g_attr_err[dev]);
@@ -260,6 +252,44 @@ ds_status fused_topk(const uint16_t* Q, const int32_t* C, const uint16_t* label,
   return launch_topk(src, idx, d.B * d.Hq, T, k, st);
 }
 
+// One-launch selection with a prefix workspace (select.cuh): r with a vector
+// path and 4096 < T <= 32768 (shorter heads are one k_topk CTA each).
+bool sel_applies(int r, int T) {
+  return (r == 8 || r == 16 || r == 32 || r == 64 || r == 128) && T > kSample && T <= kSelMaxT;
+}
+
+template <int R>
+ds_status launch_sel(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
+                     int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
+  SelParams sp;
+  sp.Q = Q;
+  sp.C = C;
+  sp.label = label;
+  sp.scores = scores;
+  sp.idx = idx;
+  sp.arrivals = static_cast<uint32_t*>(ws);
+  sp.prefixes = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kCounterBytes);
+  sp.BH = d.B * d.Hq;
+  sp.Hq = d.Hq;
+  sp.T_cap = d.T_cap;
+  sp.T = T;
+  sp.k = k;
+  dim3 grid((T + kSelTile - 1) / kSelTile, sp.BH);
+  k_score_select<R><<<grid, kSelThreads, 0, st>>>(sp);
+  return launched();
+}
+
+ds_status score_select(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
+                       int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
+  switch (d.r) {
+    case 8: return launch_sel<8>(Q, C, label, scores, idx, d, T, k, ws, st);
+    case 16: return launch_sel<16>(Q, C, label, scores, idx, d, T, k, ws, st);
+    case 32: return launch_sel<32>(Q, C, label, scores, idx, d, T, k, ws, st);
+    case 64: return launch_sel<64>(Q, C, label, scores, idx, d, T, k, ws, st);
+    default: return launch_sel<128>(Q, C, label, scores, idx, d, T, k, ws, st);
+  }
+}
+
 // Host-side check of the workspace (no CUDA calls).
 ds_status check_attend_ws(const ds_dims& d, int rows, const void* ws, size_t ws_bytes) {
   const size_t need = attend_ws_bytes(d.B * d.Hq, rows);
@@ -335,18 +365,22 @@ bool step_fused(const ds_dims& d, int T, int k, int* chunk_out, size_t* smem_out
   return true;
 }
 
-// Workspace of the separate-kernels step: the attention's split partials and
-// counters, then (when the selection runs over written scores) [BH, T] fp32
-// scores.  Returns the total; *scores_off gets the offset of the scores (0: none).
-size_t step_fallback_ws(const ds_dims& d, int T, int k, size_t* scores_off) {
+// Workspace of the separate-kernels step: the attention's counters and
+// partials, then the selection's workspace (one-launch selection) or, when the
+// selection runs over written scores, [BH, T] fp32 scores.  Returns the total;
+// *sel_off gets the offset of the second part (0: none).
+size_t step_fallback_ws(const ds_dims& d, int T, int k, size_t* sel_off) {
   const int BH = d.B * d.Hq;
   size_t n = attend_ws_bytes(BH, k);
   size_t off = 0;
-  if (prefer_score_then_select(d.r, T)) {
+  if (sel_applies(d.r, T)) {
+    off = (n + 255) & ~(size_t)255;
+    n = off + sel_ws_bytes(BH, T);
+  } else if (prefer_score_then_select(d.r, T)) {
     off = (n + 255) & ~(size_t)255;
     n = off + (((size_t)BH * T * sizeof(float) + 255) & ~(size_t)255);
   }
-  if (scores_off) *scores_off = off;
+  if (sel_off) *sel_off = off;
   return n;
 }
 
@@ -384,6 +418,9 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
       return attend_ws_bytes(BH, k);
     case DS_OP_DECODE:
       return attend_ws_bytes(BH, T);
+    case DS_OP_SCORE_TOPK:
+      if (k < 1 || k > T) return 0;
+      return sel_applies(dims.r, T) ? sel_ws_bytes(BH, T) : 0;
     case DS_OP_DECODE_STEP: {
       if (k < 1 || k > T) return 0;
       int chunk;
@@ -472,7 +509,8 @@ ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int3
 }
 
 ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, float* scores,
-                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, ds_stream_t stream) {
+                        int32_t* idx, ds_dims dims, int32_t T, int32_t k, void* ws,
+                        size_t ws_bytes, ds_stream_t stream) {
   DS_TRACE("ds_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
@@ -487,6 +525,9 @@ ds_status ds_score_topk(const void* Q, const int32_t* C, const void* label, floa
   if (s != DS_OK) return s;
   auto Qb = static_cast<const uint16_t*>(Q);
   auto Lb = static_cast<const uint16_t*>(label);
+  if (sel_applies(dims.r, T) && ws && aligned16(ws) &&
+      ws_bytes >= sel_ws_bytes(dims.B * dims.Hq, T))
+    return score_select(Qb, C, Lb, scores, idx, dims, T, k, ws, stream);
   if (scores && prefer_score_then_select(dims.r, T)) {
     s = launch_score(Qb, C, Lb, scores, dims, T, stream);
     if (s != DS_OK) return s;
@@ -692,9 +733,15 @@ ds_status decode_step(const void* Q, const void* K_new, const void* V_new, const
     s = ds_label_append(K, C, label, dims, T - 1, 1, stream);
     if (s != DS_OK) return s;
   }
-  float* scores = scores_off ? reinterpret_cast<float*>(static_cast<char*>(ws) + scores_off)
-                             : nullptr;
-  s = ds_score_topk(Q, C, label, scores, idx, dims, T, k, stream);
+  if (sel_applies(dims.r, T)) {
+    s = ds_score_topk(Q, C, label, nullptr, idx, dims, T, k, static_cast<char*>(ws) + scores_off,
+                      ws_bytes - scores_off, stream);
+  } else {
+    float* scores = prefer_score_then_select(dims.r, T)
+                        ? reinterpret_cast<float*>(static_cast<char*>(ws) + scores_off)
+                        : nullptr;
+    s = ds_score_topk(Q, C, label, scores, idx, dims, T, k, nullptr, 0, stream);
+  }
   if (s != DS_OK) return s;
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
 }

@@ -1,0 +1,512 @@
+// Per-head top-k for heads of moderate length (4096 < T <= 32768), from the
+// label cache, in one launch with a workspace.
+//
+// Token selection keeps the tokens with the highest approximate activation
+// (Double Sparsity, Method details: Key design); contract as for k_topk: the k
+// largest scores, ties to the lower token index, -0 == +0, output ascending.
+//
+// Grid (tiles, heads): each CTA streams one tile of kSelTile tokens of one
+// head's label rows (the HBM-bound part), computes every token's fp32 score
+// exactly as k_score_vec does (optionally writing it out) and stores only the
+// top 16 bits of its order-preserving key in the workspace (2 bytes a token).
+// The head's last tile to finish (a per-head arrival counter) then selects the
+// head from those prefixes, which are still in L2, while other CTAs keep
+// streaming:
+//   1. a bracket [lo, hi] on the prefixes from a 2048-token subsample (ranks
+//      k*m/T -/+ (5 sd + 2), as k_topk brackets its sample);
+//   2. one pass over each thread's run of tokens builds two register bit
+//      masks: above the bracket, and inside it (the candidates);
+//   3. the candidates (token order) give the 16-bit bin B16 of the k-th key;
+//   4. B16's tokens have their exact keys recomputed from their label rows and
+//      a radix select over the keys' low 16 bits gives the exact threshold;
+//      kept tokens of B16 are marked, ties in token order up to the rank needed;
+//   5. each thread writes its kept tokens, ascending.
+// The prefixes' L2 lines are then discarded (no write-back of a buffer that is
+// dead).  When the bracket misses, histograms of every prefix give B16 instead; when
+// B16 holds more tokens than its list, their exact keys are recomputed in
+// place (both slower, both exact).
+#pragma once
+
+#include "topk.cuh"
+
+namespace ds {
+
+constexpr int kSelThreads = kTopkThreads;  // 8 warps: LabelSource's slicing
+constexpr int kSelTile = 16384;            // tokens scored by one CTA
+constexpr int kSelMaxT = 32768;            // 128 tokens per selector thread at most
+constexpr int kSelMaxRun = kSelMaxT / kSelThreads;
+constexpr int kSelListCap = 2048;          // candidates (and B16's tokens) held in lists
+constexpr int kSelSample = 2048;           // prefixes sampled for the bracket
+constexpr int kSelSlots = 8;               // label loads in flight per thread
+static_assert(kSelThreads == 256, "the selector's scans and 256-bin histograms take 256 threads");
+
+// Tokens of each selector thread: a power of two >= T/256 (at least 8: whole
+// 16-byte prefix runs), so that a token's place is found by shifts.
+__host__ __device__ inline int sel_per(int T) {
+  int per = 8;
+  while (per * kSelThreads < T) per <<= 1;
+  return per;
+}
+__host__ __device__ inline int sel_tpad(int T) { return sel_per(T) * kSelThreads; }
+
+// Workspace: one arrival counter per head at a fixed place (zero between
+// calls), then each head's prefixes, T_pad 16-bit words.
+__host__ __device__ inline size_t sel_ws_bytes(int BH, int T) {
+  const size_t b = kCounterBytes + (size_t)BH * sel_tpad(T) * 2;
+  return (b + 255) & ~size_t(255);
+}
+
+// Prefixes are stored transposed: selector thread ct owns tokens
+// [ct*per, (ct+1)*per), and its i-th run of 8 sits in 16-byte word
+// i*256 + ct, so that a warp's 16-byte loads are consecutive.  Index of token
+// t's prefix, in 16-bit units.
+__device__ __forceinline__ int key_slot(int t, int per) {
+  const int lg = 31 - __clz(per);
+  const int ct = t >> lg, j = t & (per - 1);
+  return (((j >> 3) * kSelThreads + ct) << 3) + (j & 7);
+}
+
+struct SelParams {
+  const uint16_t* Q;
+  const int32_t* C;
+  const uint16_t* label;
+  float* scores;        // optional [BH, T]
+  int32_t* idx;         // [BH, k]
+  uint32_t* arrivals;   // [BH]
+  uint16_t* prefixes;   // [BH, T_pad]
+  int BH, Hq, T_cap, T, k;
+};
+
+enum { S_BIN = 0, S_ABV = 1, S_CNT = 2, S_LAST = 3 };
+
+// The fp32 score of one label row computed by one thread in exactly the order
+// of lane_group_score: 8-channel chunk sums, then pairwise as the butterfly
+// adds them.
+template <int R>
+__device__ __forceinline__ float exact_row_score(const uint16_t* row, const float* qs) {
+  constexpr int NC = R / 8;
+  float a[NC];
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) a[c] = chunk_dot(__ldg(r4 + c), qs + 8 * c);
+#pragma unroll
+  for (int st = 1; st < NC; st <<= 1)
+#pragma unroll
+    for (int i = 0; i < NC; i += 2 * st) a[i] = a[i] + a[i + st];
+  return a[0];
+}
+
+// Exact keys of the n tokens tok[0..n) into key[], the CTA's threads taking
+// items tid, tid+256, ...: a batch of items' label rows is loaded before any
+// is used, so that their loads are in flight together.
+template <int R>
+__device__ __forceinline__ void exact_keys(const uint16_t* lab, const float* qs,
+                                           const uint32_t* tok, uint32_t* key, int n) {
+  constexpr int NC = R / 8;
+  constexpr int kBatch = NC >= 8 ? 1 : 8 / NC;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kBatch * kSelThreads) {
+    uint4 x[kBatch][NC];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = i0 + b * kSelThreads;
+      const uint4* r4 = reinterpret_cast<const uint4*>(lab + (size_t)(i < n ? tok[i] : 0) * R);
+#pragma unroll
+      for (int c = 0; c < NC; ++c) x[b][c] = i < n ? __ldg(r4 + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = i0 + b * kSelThreads;
+      float a[NC];
+#pragma unroll
+      for (int c = 0; c < NC; ++c) a[c] = chunk_dot(x[b][c], qs + 8 * c);
+#pragma unroll
+      for (int st = 1; st < NC; st <<= 1)
+#pragma unroll
+        for (int j = 0; j < NC; j += 2 * st) a[j] = a[j] + a[j + st];
+      if (i < n) key[i] = order_key(a[0]);
+    }
+  }
+}
+
+// Inclusive prefix over the CTA's threads in order; *total: the sum.
+// scratch: 8 words, not rewritten before the caller's next barrier.
+__device__ __forceinline__ uint32_t blk_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) scratch[w] = incl;
+  __syncthreads();
+  uint32_t base = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < kSelThreads / 32; ++i) {
+    const uint32_t x = scratch[i];
+    if (i < w) base += x;
+    tot += x;
+  }
+  *total = tot;
+  return base + incl;
+}
+
+// In a 256-bin histogram (bins counted from the top), the bin b holding rank r
+// (1 = largest): misc[S_BIN] = b, misc[S_ABV] = count above it, misc[S_CNT] =
+// its count.  Ends with a barrier.
+__device__ __forceinline__ void blk_find_bin(const uint32_t* hist, uint32_t r, uint32_t* scratch,
+                                             uint32_t* misc) {
+  const uint32_t c = hist[255 - threadIdx.x];
+  uint32_t tot;
+  const uint32_t incl = blk_scan(c, scratch, &tot);
+  if (c > 0 && incl - c < r && r <= incl) {
+    misc[S_BIN] = 255u - threadIdx.x;
+    misc[S_ABV] = incl - c;
+    misc[S_CNT] = c;
+  }
+  __syncthreads();
+}
+
+// The 16-bit key of rank r among n keys (key_of(i) & 0xffff, i < n) by two
+// 8-bit histogram levels; *above / *eq: counts above and equal to it.
+template <class KeyOf>
+__device__ __forceinline__ uint32_t blk_select16(KeyOf key_of, int n, uint32_t r, uint32_t* hist,
+                                                 uint32_t* scratch, uint32_t* misc,
+                                                 uint32_t* above, uint32_t* eq) {
+  hist[threadIdx.x] = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kSelThreads)
+    atomicAdd(&hist[(key_of(i) >> 8) & 255u], 1u);
+  __syncthreads();
+  blk_find_bin(hist, r, scratch, misc);
+  const uint32_t b1 = misc[S_BIN], a1 = misc[S_ABV];
+  hist[threadIdx.x] = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t key = key_of(i) & 0xffffu;
+    if ((key >> 8) == b1) atomicAdd(&hist[key & 255u], 1u);
+  }
+  __syncthreads();
+  blk_find_bin(hist, r - a1, scratch + 8, misc);
+  *above = a1 + misc[S_ABV];
+  *eq = misc[S_CNT];
+  return (b1 << 8) | misc[S_BIN];
+}
+
+// Calls f(j, prefix) for j = 0 .. per-1 of this thread's run (j: the token's
+// offset in the run), eight prefixes per 16-byte load, read around L1 (the
+// prefixes were written by other CTAs).
+template <class F>
+__device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f) {
+  const uint4* p4 = reinterpret_cast<const uint4*>(pref);
+#pragma unroll
+  for (int i = 0; i < kSelMaxRun / 8; ++i) {
+    if (i < per / 8) {
+      const uint4 v = __ldcg(p4 + i * kSelThreads + threadIdx.x);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f(8 * i + e, (w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+    }
+  }
+}
+
+struct SelSmem {
+  float qs[128];
+  uint32_t hist[256];
+  uint32_t misc[8];
+  uint32_t scan[16];
+  uint16_t smp[kSelSample];  // the bracket's subsample of prefixes
+  uint32_t ltok[kSelListCap];
+  uint32_t lkey[kSelListCap];
+  uint32_t selb[kSelMaxT / 32];  // kept tokens found through the lists
+};
+
+// Selection of head bh from its prefixes, by the whole CTA.
+template <int R>
+__device__ void select_head(const SelParams& p, int bh, SelSmem& s) {
+  const int T = p.T, per = sel_per(T), tp = per * kSelThreads;
+  const int t0 = threadIdx.x * per;
+  const uint16_t* pref = p.prefixes + (size_t)bh * tp;
+  const uint16_t* lab = p.label + (size_t)bh * p.T_cap * R;
+  const uint32_t k = (uint32_t)p.k;
+  auto exact_key = [&](int t) { return order_key(exact_row_score<R>(lab + (size_t)t * R, s.qs)); };
+  auto in_t = [&](int j) { return t0 + j < T; };
+
+  for (int i = threadIdx.x; i < tp / 32; i += kSelThreads) s.selb[i] = 0u;
+
+  // 1. bracket from a subsample of the prefixes
+  const int stride = tp / kSelSample;
+  const int mv = (T + stride - 1) / stride;  // sampled tokens below T
+  const float e = (float)k * (float)mv / (float)T;
+  const float sd = sqrtf(e * (1.f - (float)k / (float)T));
+  const float margin = kBracketSigmas * sd + 2.f;
+  const int r_hi = (int)floorf(e - margin), r_lo = (int)ceilf(e + margin);
+  // the subsample in shared memory (one batch of loads)
+  {
+    uint16_t v[kSelSample / kSelThreads];
+#pragma unroll
+    for (int j = 0; j < kSelSample / kSelThreads; ++j) {
+      const int i = threadIdx.x + j * kSelThreads;
+      v[j] = i < mv ? __ldcg(pref + key_slot(i * stride, per)) : (uint16_t)0;
+    }
+#pragma unroll
+    for (int j = 0; j < kSelSample / kSelThreads; ++j) s.smp[threadIdx.x + j * kSelThreads] = v[j];
+  }
+  __syncthreads();
+  auto sample = [&](int i) { return (uint32_t)s.smp[i]; };
+  uint32_t hi = 0xffffffffu, lo = 0u, ua, ue;
+  if (r_hi >= 1) hi = blk_select16(sample, mv, (uint32_t)r_hi, s.hist, s.scan, s.misc, &ua, &ue);
+  if (r_lo <= mv) lo = blk_select16(sample, mv, (uint32_t)r_lo, s.hist, s.scan, s.misc, &ua, &ue);
+
+  // 2. register masks of this thread's run: above the bracket, inside it
+  uint32_t am[4] = {0u, 0u, 0u, 0u}, cm[4] = {0u, 0u, 0u, 0u};
+  for_my_run(pref, per, [&](int j, uint32_t key) {
+    const bool v = in_t(j);
+    am[j >> 5] |= (uint32_t)(v && key > hi) << (j & 31);
+    cm[j >> 5] |= (uint32_t)(v && key >= lo && key <= hi) << (j & 31);
+  });
+  const uint32_t na = __popc(am[0]) + __popc(am[1]) + __popc(am[2]) + __popc(am[3]);
+  const uint32_t nc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
+  uint32_t tot;
+  const uint32_t incl = blk_scan(na | (nc << 16), s.scan, &tot);
+  const uint32_t n_above = tot & 0xffffu, n_cand = tot >> 16;
+  const bool listed = n_cand <= (uint32_t)kSelListCap && n_above < k && k <= n_above + n_cand;
+  __syncthreads();
+
+  // 3. the bin B16 of the k-th key
+  uint32_t B16, ngt16, neq;
+  if (listed) {
+    // the candidates in token order: the 16-byte prefix words that hold any are
+    // loaded again, all at once
+    uint32_t pos = (incl - (na | (nc << 16))) >> 16;
+    const uint4* p4 = reinterpret_cast<const uint4*>(pref);
+#pragma unroll
+    for (int i = 0; i < kSelMaxRun / 8; ++i) {
+      const uint32_t bits8 = (cm[i >> 2] >> (8 * (i & 3))) & 255u;
+      if (i < per / 8 && bits8) {
+        const uint4 v = __ldcg(p4 + i * kSelThreads + threadIdx.x);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) {
+          if ((bits8 >> e8) & 1u) {
+            s.ltok[pos] = (uint32_t)(t0 + 8 * i + e8);
+            s.lkey[pos] = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xffffu;
+            ++pos;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    uint32_t above_c;
+    B16 = blk_select16([&](int i) { return s.lkey[i]; }, (int)n_cand, k - n_above, s.hist,
+                       s.scan, s.misc, &above_c, &neq);
+    ngt16 = n_above + above_c;
+    // candidates above B16 join the bitmap
+    for (uint32_t i = threadIdx.x; i < n_cand; i += kSelThreads) {
+      const uint32_t t = s.ltok[i];
+      if (s.lkey[i] > B16) atomicOr(&s.selb[t >> 5], 1u << (t & 31));
+    }
+  } else {
+    // the bracket missed: histograms of every prefix
+    s.hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for_my_run(pref, per, [&](int j, uint32_t key) {
+      if (in_t(j)) atomicAdd(&s.hist[key >> 8], 1u);
+    });
+    __syncthreads();
+    blk_find_bin(s.hist, k, s.scan, s.misc);
+    const uint32_t b1 = s.misc[S_BIN], a1 = s.misc[S_ABV];
+    s.hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for_my_run(pref, per, [&](int j, uint32_t key) {
+      if (in_t(j) && (key >> 8) == b1) atomicAdd(&s.hist[key & 255u], 1u);
+    });
+    __syncthreads();
+    blk_find_bin(s.hist, k - a1, s.scan + 8, s.misc);
+    B16 = (b1 << 8) | s.misc[S_BIN];
+    ngt16 = a1 + s.misc[S_ABV];
+    neq = s.misc[S_CNT];
+    // this thread's tokens above B16
+    am[0] = am[1] = am[2] = am[3] = 0u;
+    for_my_run(pref, per, [&](int j, uint32_t key) {
+      am[j >> 5] |= (uint32_t)(in_t(j) && key > B16) << (j & 31);
+    });
+  }
+  __syncthreads();
+
+  // 4. B16's tokens: all kept, or the exact threshold among them
+  const uint32_t need = k - ngt16;  // 1 <= need <= neq
+  uint32_t bm[4] = {0u, 0u, 0u, 0u};  // this thread's tokens of B16
+  if (listed) {
+    // B16 lies inside the bracket: its tokens are candidates of this thread's
+    // own run, in the list slice this thread wrote
+    const uint32_t pos0 = (incl - (na | (nc << 16))) >> 16;
+    for (uint32_t i = pos0; i < pos0 + nc; ++i)
+      if (s.lkey[i] == B16) {
+        const int j = (int)s.ltok[i] - t0;
+        bm[j >> 5] |= 1u << (j & 31);
+      }
+  } else {
+    for_my_run(pref, per, [&](int j, uint32_t key) {
+      bm[j >> 5] |= (uint32_t)(in_t(j) && key == B16) << (j & 31);
+    });
+  }
+  if (need == neq) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) am[w] |= bm[w];
+  } else if (neq <= (uint32_t)kSelListCap) {
+    // B16's tokens in token order, their exact keys, the threshold over the
+    // keys' low 16 bits, then the kept ones (ties in order up to the rank needed)
+    const uint32_t nb = __popc(bm[0]) + __popc(bm[1]) + __popc(bm[2]) + __popc(bm[3]);
+    uint32_t pos = blk_scan(nb, s.scan, &tot) - nb;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        s.ltok[pos++] = (uint32_t)(t0 + 32 * w + __ffs(bits) - 1);
+        bits &= bits - 1u;
+      }
+    }
+    __syncthreads();
+    exact_keys<R>(lab, s.qs, s.ltok, s.lkey, (int)neq);
+    __syncthreads();
+    uint32_t above_e, eq_e;
+    const uint32_t thr =
+        (B16 << 16) | blk_select16([&](int i) { return s.lkey[i]; }, (int)neq, need, s.hist,
+                                   s.scan, s.misc, &above_e, &eq_e);
+    const uint32_t need_eq = need - above_e;
+    const int per_t = ((int)neq + kSelThreads - 1) / kSelThreads;
+    const int s0 = min((int)threadIdx.x * per_t, (int)neq), s1 = min(s0 + per_t, (int)neq);
+    uint32_t nt = 0;
+    for (int i = s0; i < s1; ++i) nt += s.lkey[i] == thr;
+    uint32_t rank = blk_scan(nt, s.scan, &tot) - nt;
+    for (int i = s0; i < s1; ++i) {
+      const uint32_t key = s.lkey[i], t = s.ltok[i];
+      bool keep = key > thr;
+      if (key == thr) keep = rank++ < need_eq;
+      if (keep) atomicOr(&s.selb[t >> 5], 1u << (t & 31));
+    }
+  } else {
+    // more tokens in B16 than the list holds: exact keys recomputed in place
+    uint32_t rank = need, pf = 0u;
+    for (int d = 0; d < 2; ++d) {
+      s.hist[threadIdx.x] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t bits = bm[w];
+        while (bits) {
+          const uint32_t key = exact_key(t0 + 32 * w + __ffs(bits) - 1);
+          bits &= bits - 1u;
+          if (d == 0)
+            atomicAdd(&s.hist[(key >> 8) & 255u], 1u);
+          else if (((key >> 8) & 255u) == pf)
+            atomicAdd(&s.hist[key & 255u], 1u);
+        }
+      }
+      __syncthreads();
+      blk_find_bin(s.hist, rank, s.scan + 8 * d, s.misc);
+      rank -= s.misc[S_ABV];
+      pf = d == 0 ? s.misc[S_BIN] : (pf << 8) | s.misc[S_BIN];
+    }
+    const uint32_t thr = (B16 << 16) | pf, need_eq = rank;
+    // ties in token order: this thread's count first
+    uint32_t nt = 0, gtw[4] = {0u, 0u, 0u, 0u}, eqw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int j = 32 * w + __ffs(bits) - 1;
+        bits &= bits - 1u;
+        const uint32_t key = exact_key(t0 + j);
+        gtw[w] |= (uint32_t)(key > thr) << (j & 31);
+        eqw[w] |= (uint32_t)(key == thr) << (j & 31);
+      }
+      nt += __popc(eqw[w]);
+    }
+    uint32_t rk = blk_scan(nt, s.scan, &tot) - nt;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      am[w] |= gtw[w];
+      uint32_t bits = eqw[w];
+      while (bits) {
+        const int j = 32 * w + __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (rk++ < need_eq) am[w] |= 1u << (j & 31);
+      }
+    }
+  }
+  __syncthreads();
+
+  // the prefixes are read for the last time: drop their L2 lines without
+  // writing them back (the next call writes them again)
+  {
+    const char* pb = reinterpret_cast<const char*>(pref);
+    if ((reinterpret_cast<uintptr_t>(pb) & 127) == 0)  // whole 128-byte lines only
+      for (int i = threadIdx.x; i < tp * 2 / 128; i += kSelThreads)
+        asm volatile("discard.global.L2 [%0], 128;" ::"l"(pb + (size_t)i * 128) : "memory");
+  }
+
+  // 5. write this thread's kept tokens, ascending
+  uint32_t sel[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t m = 0u;
+    if (per >= 32) {
+      if (32 * w < per) m = s.selb[(t0 >> 5) + w];
+    } else if (w == 0) {
+      m = (s.selb[t0 >> 5] >> (t0 & 31)) & ((1u << per) - 1u);
+    }
+    sel[w] = am[w] | m;
+  }
+  const uint32_t cnt = __popc(sel[0]) + __popc(sel[1]) + __popc(sel[2]) + __popc(sel[3]);
+  uint32_t out = blk_scan(cnt, s.scan, &tot) - cnt;
+  int32_t* dst = p.idx + (size_t)bh * p.k;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t bits = sel[w];
+    while (bits) {
+      const int t = t0 + 32 * w + __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (out < k) dst[out] = t;
+      ++out;
+    }
+  }
+}
+
+// grid (ceil(T / kSelTile), BH), kSelThreads threads.
+template <int R>
+__global__ void __launch_bounds__(kSelThreads, 3)
+k_score_select(const SelParams p) {
+  __shared__ SelSmem s;
+  const int bh = blockIdx.y;
+  const int per = sel_per(p.T);
+  const int tile0 = blockIdx.x * kSelTile;
+  const int n = min(kSelTile, p.T - tile0);
+  uint16_t* pref = p.prefixes + (size_t)bh * per * kSelThreads;
+  float* so = p.scores ? p.scores + (size_t)bh * p.T : nullptr;
+
+  LabelSource<R, kSelSlots> src{p.Q, p.C, p.label, nullptr, p.Hq, p.T_cap};
+  src.prepare(bh, s.qs);
+  __syncthreads();
+  src.stream(bh, p.T, n, [tile0](int j) { return tile0 + j; },
+             [&](bool v, int j, uint32_t key, float sc) {
+               if (v) {
+                 pref[key_slot(tile0 + j, per)] = (uint16_t)(key >> 16);
+                 if (so) so[tile0 + j] = sc;
+               }
+             },
+             s.qs);
+  // the head's last tile to finish selects it
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    s.misc[S_LAST] = atomicAdd(&p.arrivals[bh], 1u) == gridDim.x - 1 ? 1u : 0u;
+  __syncthreads();
+  if (s.misc[S_LAST] == 0u) return;
+  __threadfence();
+  select_head<R>(p, bh, s);
+  if (threadIdx.x == 0) p.arrivals[bh] = 0u;  // zero again for the next call
+}
+
+}  // namespace ds

@@ -73,7 +73,7 @@ def test_bad_dims(dims, want):
     d = _dims(**dims)
     assert lib.ds_label_append(P, P, P, d, 0, 1, NUL) == want
     assert lib.ds_score(P, P, P, P, d, 10, NUL) == want
-    assert lib.ds_score_topk(P, P, P, NUL, P, d, 10, 5, NUL) == want
+    assert lib.ds_score_topk(P, P, P, NUL, P, d, 10, 5, NUL, 0, NUL) == want
     assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 10, 5, 1.0, NUL, 0, NUL) == want
     assert lib.ds_decode(P, P, P, P, NUL, d, 10, 1.0, NUL, 0, NUL) == want
 
@@ -102,8 +102,9 @@ def test_bad_sizes_and_pointers():
     assert lib.ds_topk(P, P, 4, 16 * 65536 + 1, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
     assert lib.ds_topk(P, P, 70000, 10, 1, NUL, 0, NUL) == ds.DS_ERR_UNSUPPORTED
     # fused score+topk: r not a multiple of 8 needs a score buffer
-    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 20, NUL) == bad
-    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 5, NUL) == ds.DS_ERR_UNSUPPORTED
+    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 20, NUL, 0, NUL) == bad
+    assert lib.ds_score_topk(P, P, P, NUL, P, _dims(r=5), 10, 5, NUL, 0, NUL) == \
+        ds.DS_ERR_UNSUPPORTED
     # sparse decode: k > T, T > T_cap, misaligned lse
     assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 10, 11, 1.0, NUL, 0, NUL) == bad
     assert lib.ds_sparse_decode(P, P, P, P, P, NUL, d, 1001, 5, 1.0, NUL, 0, NUL) == bad
@@ -131,7 +132,13 @@ def test_workspace_sizes():
     d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
     assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 16) == 0
     assert lib.ds_workspace_size(ds.OP_TOPK, d, 32768, 512) == 0
-    assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == 0
+    # the one-launch selection keeps 2-byte key prefixes of every token (T_pad a
+    # power of two times 256) after 256 KiB of counters
+    assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == \
+        256 * 1024 + 32 * 32 * 32768 * 2
+    assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 4096, 512) == 0  # one CTA per head
+    assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 5000, 512) == \
+        256 * 1024 + 32 * 32 * 8192 * 2
     # heads shared by warps: 256 KiB of counters, then 132 floats per slot
     n = lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 2048)
     assert n > 256 * 1024 and n % 256 == 0
