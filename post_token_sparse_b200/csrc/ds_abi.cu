@@ -16,6 +16,7 @@
 #include "ds.h"
 
 #include "attend.cuh"
+#include "attend_group.cuh"
 #include "calib.cuh"
 #include "common.cuh"
 #include "label.cuh"
@@ -106,6 +107,19 @@ ds_status check_dims(const ds_dims& d) {
 // fixed place, then the partials of the heads that several warps share.
 size_t attend_ws_bytes(int heads, int rows) { return attn_workspace_bytes(attn_plan(heads, rows)); }
 
+// Attention over rows shared by a whole group of query heads (all T tokens, or
+// a group-shared token set) runs group by group (k_attend_group) when a KV head
+// has 2..8 query heads, else head by head.
+bool group_kernel_applies(const ds_dims& d) {
+  const int G = d.Hq / d.Hkv;
+  return G >= 2 && G <= kGrpMaxG;
+}
+// workspace of an attention call whose rows are shared by each group
+size_t shared_rows_ws_bytes(const ds_dims& d, int rows) {
+  if (group_kernel_applies(d)) return grp_workspace_bytes(grp_plan(d.B * d.Hkv, rows));
+  return attend_ws_bytes(d.B * d.Hq, rows);
+}
+
 // ---- per-device one-time kernel attributes ----------------------------------
 constexpr int kMaxDevices = 64;
 std::once_flag g_attr_once[kMaxDevices];
@@ -136,6 +150,8 @@ ds_status ensure_attrs() {
     };
     acc(allow_smem(k_attend<true>, kAttnSmemBytes));
     acc(allow_smem(k_attend<false>, kAttnSmemBytes));
+    acc(allow_smem(k_attend_group<true>, kGrpSmemBytes));
+    acc(allow_smem(k_attend_group<false>, kGrpSmemBytes));
     acc(topk_attrs<ScoresSource>());
     acc(topk_attrs<LabelSource<8>>());
     acc(topk_attrs<LabelSource<16>>());
@@ -279,6 +295,33 @@ ds_status launch_sel(const uint16_t* Q, const int32_t* C, const uint16_t* label,
   return launched();
 }
 
+// One-launch group selection: as sel_applies, with the group's query values
+// (G * r floats) in the CTA's shared memory.
+bool grp_sel_applies(const ds_dims& d, int T) {
+  return sel_applies(d.r, T) && (d.Hq / d.Hkv) * d.r <= kGrpSelMaxQ;
+}
+
+template <int R>
+ds_status launch_grp_sel(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* sg,
+                         int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
+  SelParams sp;
+  sp.Q = Q;
+  sp.C = C;
+  sp.label = label;
+  sp.scores = sg;
+  sp.idx = idx;
+  sp.arrivals = static_cast<uint32_t*>(ws);
+  sp.prefixes = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kCounterBytes);
+  sp.BH = d.B * d.Hkv;
+  sp.Hq = d.Hq;
+  sp.T_cap = d.T_cap;
+  sp.T = T;
+  sp.k = k;
+  dim3 grid((T + kGrpSelTile - 1) / kGrpSelTile, sp.BH);
+  k_group_score_select<R><<<grid, kSelThreads, 0, st>>>(sp, d.Hkv);
+  return launched();
+}
+
 ds_status score_select(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
                        int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
   switch (d.r) {
@@ -295,6 +338,48 @@ ds_status check_attend_ws(const ds_dims& d, int rows, const void* ws, size_t ws_
   const size_t need = attend_ws_bytes(d.B * d.Hq, rows);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return DS_ERR_WORKSPACE;
   return DS_OK;
+}
+
+// Host-side check of the workspace of a call whose rows each group shares.
+ds_status check_shared_rows_ws(const ds_dims& d, int rows, const void* ws, size_t ws_bytes) {
+  const size_t need = shared_rows_ws_bytes(d, rows);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return DS_ERR_WORKSPACE;
+  return DS_OK;
+}
+
+// Group-by-group attention (group_kernel_applies): idx [B*Hkv, rows] shared
+// token ids, or null for all T tokens.
+ds_status launch_attend_group(const ds_dims& d, const void* Q, const void* K, const void* V,
+                              const int32_t* idx, float* O, float* lse, int T, int rows,
+                              float scale, void* ws, cudaStream_t st) {
+  const int groups = d.B * d.Hkv;
+  const AttnPlan pl = grp_plan(groups, rows);
+  GrpParams p;
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.idx = idx;
+  p.O = O;
+  p.lse = lse;
+  p.arrivals = pl.slots ? static_cast<uint32_t*>(ws) : nullptr;
+  p.partial = pl.slots ? reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes)
+                       : nullptr;
+  p.groups = groups;
+  p.G = d.Hq / d.Hkv;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.T_cap = d.T_cap;
+  p.T = T;
+  p.rows = rows;
+  p.per = pl.per;
+  p.units = pl.units;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int grid = (pl.units + kGrpWarps - 1) / kGrpWarps;
+  if (idx)
+    k_attend_group<true><<<grid, kGrpThreads, kGrpSmemBytes, st>>>(p);
+  else
+    k_attend_group<false><<<grid, kGrpThreads, kGrpSmemBytes, st>>>(p);
+  return launched();
 }
 
 ds_status launch_attend(const ds_dims& d, const void* Q, const void* K, const void* V,
@@ -417,7 +502,7 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
       if (k < 1 || k > T) return 0;
       return attend_ws_bytes(BH, k);
     case DS_OP_DECODE:
-      return attend_ws_bytes(BH, T);
+      return shared_rows_ws_bytes(dims, T);
     case DS_OP_SCORE_TOPK:
       if (k < 1 || k > T) return 0;
       return sel_applies(dims.r, T) ? sel_ws_bytes(BH, T) : 0;
@@ -431,9 +516,12 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
     case DS_OP_BLOCK_SPARSE_DECODE:  // k: kept rows, blocks x block size
       if (k < 1) return 0;
       return attend_ws_bytes(BH, k);
-    case DS_OP_GROUP_SPARSE_DECODE:  // the same plan as the per-head call
+    case DS_OP_GROUP_SPARSE_DECODE:
       if (k < 1 || k > T) return 0;
-      return attend_ws_bytes(BH, k);
+      return shared_rows_ws_bytes(dims, k);
+    case DS_OP_GROUP_SCORE_TOPK:
+      if (k < 1 || k > T) return 0;
+      return grp_sel_applies(dims, T) ? sel_ws_bytes(dims.B * dims.Hkv, T) : 0;
     case DS_OP_CALIBRATE: {
       if (k < 1) return 0;  // k: calibration queries per head
       const size_t nck = (T + kAbsumRows - 1) / kAbsumRows, ncq = (k + kAbsumRows - 1) / kAbsumRows;
@@ -576,12 +664,14 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
       !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap) return DS_ERR_INVALID_ARG;
-  s = check_attend_ws(dims, T, ws, ws_bytes);
+  s = check_shared_rows_ws(dims, T, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
+  if (group_kernel_applies(dims))
+    return launch_attend_group(dims, Q, K, V, nullptr, O, lse, T, T, scale, ws, stream);
   return launch_attend(dims, Q, K, V, nullptr, O, lse, T, T, scale, ws, stream);
 }
 
@@ -816,7 +906,8 @@ ds_status launch_group_score(const uint16_t* Q, const int32_t* C, const uint16_t
 
 extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
                                          float* group_scores, int32_t* idx, ds_dims dims,
-                                         int32_t T, int32_t k, ds_stream_t stream) {
+                                         int32_t T, int32_t k, void* ws, size_t ws_bytes,
+                                         ds_stream_t stream) {
   DS_TRACE("ds_group_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
@@ -833,6 +924,16 @@ extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const 
   if (s != DS_OK) return s;
   auto Qb = static_cast<const uint16_t*>(Q);
   auto Lb = static_cast<const uint16_t*>(label);
+  if (grp_sel_applies(dims, T) && ws && aligned16(ws) &&
+      ws_bytes >= sel_ws_bytes(dims.B * dims.Hkv, T)) {
+    switch (dims.r) {
+      case 8: return launch_grp_sel<8>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
+      case 16: return launch_grp_sel<16>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
+      case 32: return launch_grp_sel<32>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
+      case 64: return launch_grp_sel<64>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
+      default: return launch_grp_sel<128>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
+    }
+  }
   switch (dims.r) {
     case 8: s = launch_group_score<8>(Qb, C, Lb, group_scores, dims, T, stream); break;
     case 16: s = launch_group_score<16>(Qb, C, Lb, group_scores, dims, T, stream); break;
@@ -856,12 +957,14 @@ extern "C" ds_status ds_group_sparse_decode(const void* Q, const void* K, const 
       !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
     return DS_ERR_INVALID_ARG;
   if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
-  s = check_attend_ws(dims, k, ws, ws_bytes);
+  s = check_shared_rows_ws(dims, k, ws, ws_bytes);
   if (s != DS_OK) return s;
   s = check_kv(K, V);
   if (s != DS_OK) return s;
   s = ensure_attrs();
   if (s != DS_OK) return s;
+  if (group_kernel_applies(dims))
+    return launch_attend_group(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream, true);
 }
 

@@ -152,19 +152,29 @@ k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
            lane / S::kLanes;
   };
   float acc[S::kSlots];
-  for (int hh = 0; hh < G; ++hh) {
-    const uint4* lab =
+  // two heads' rows loaded before either is used (twice the loads in flight)
+  for (int hh = 0; hh < G; hh += 2) {
+    const bool two = hh + 1 < G;
+    const uint4* lab0 =
         reinterpret_cast<const uint4*>(label + (size_t)(b * Hq + g * G + hh) * T_cap * R);
-    uint4 v[S::kSlots];
+    const uint4* lab1 = lab0 + (size_t)T_cap * S::kLanes;
+    uint4 v0[S::kSlots], v1[S::kSlots];
 #pragma unroll
     for (int i = 0; i < S::kSlots; ++i) {
       const int t = token(i);
-      v[i] = t < T ? ldg_stream(lab + (size_t)t * S::kLanes + chunk) : make_uint4(0, 0, 0, 0);
+      v0[i] = t < T ? ldg_stream(lab0 + (size_t)t * S::kLanes + chunk) : make_uint4(0, 0, 0, 0);
+      v1[i] = two && t < T ? ldg_stream(lab1 + (size_t)t * S::kLanes + chunk)
+                           : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int i = 0; i < S::kSlots; ++i) {
-      const float s = lane_group_score<R>(v[i], qg + hh * R, chunk);  // all lanes take part
-      acc[i] = hh == 0 ? s : acc[i] + s;
+      // head order: acc + s(hh), then + s(hh+1); all lanes take part
+      const float s0 = lane_group_score<R>(v0[i], qg + hh * R, chunk);
+      acc[i] = hh == 0 ? s0 : acc[i] + s0;
+      if (two) {
+        const float s1 = lane_group_score<R>(v1[i], qg + (hh + 1) * R, chunk);
+        acc[i] = acc[i] + s1;
+      }
     }
   }
   float* out = sg + (size_t)bg * T;

@@ -169,25 +169,38 @@ def test_decode_step_fuses_only_one_wave_of_heads():
                                  32768, 2048) > 0
 
 
+def test_group_score_topk_workspace():
+    """One-launch group selection for 4096 < T <= 32768 and G*r <= 1024: the
+    arrival counters, then 16-bit prefixes of every group's padded T."""
+    lib = ds.lib()
+    d = _dims(B=16, Hq=64, Hkv=8, T_cap=16384, r=16)
+    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, d, 16384, 1024) == \
+        256 * 1024 + 128 * 16384 * 2
+    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, d, 4096, 100) == 0
+    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, _dims(B=1, Hq=64, Hkv=4, T_cap=9000,
+                                                               r=128), 9000, 10) == 0
+
+
 def test_group_calls_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG
     d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
     mis = ctypes.c_void_p(FAKE + 4)
-    assert lib.ds_group_score_topk(P, P, P, NUL, P, d, 100, 10, NUL) == bad  # scores required
-    assert lib.ds_group_score_topk(P, P, P, P, P, d, 100, 101, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, d, 1001, 10, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, mis, P, d, 100, 10, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(Hq=6, Hkv=4), 100, 10, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(r=12), 100, 10, NUL) == \
+    assert lib.ds_group_score_topk(P, P, P, NUL, P, d, 100, 10, NUL, 0, NUL) == bad  # scores required
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 100, 101, NUL, 0, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 1001, 10, NUL, 0, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, mis, P, d, 100, 10, NUL, 0, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(Hq=6, Hkv=4), 100, 10, NUL, 0, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(r=12), 100, 10, NUL, 0, NUL) == \
         ds.DS_ERR_UNSUPPORTED
     assert lib.ds_group_sparse_decode(P, P, P, P, P, NUL, d, 100, 101, 1.0, NUL, 0, NUL) == bad
     assert lib.ds_group_sparse_decode(P, P, P, NUL, P, NUL, d, 100, 10, 1.0, NUL, 0, NUL) == bad
-    # the same split plan (and workspace) as the per-head attention
+    # G = 4: the group-by-group plan over the 8 groups' shared rows
     dl = _dims(B=1, Hq=32, Hkv=8, T_cap=262144, r=8)
-    assert lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384) == \
-        lib.ds_workspace_size(ds.OP_SPARSE_DECODE, dl, 262144, 16384) > 0
+    slots = _group_plan(8, 16384)
+    assert slots > 0
     need = lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384)
+    assert need == (256 * 1024 + slots * 8 * 132 * 4 + 255) // 256 * 256
     assert lib.ds_group_sparse_decode(P, P, P, P, P, NUL, dl, 262144, 16384, 1.0, P, need - 1,
                                       NUL) == ds.DS_ERR_WORKSPACE
 
@@ -313,6 +326,40 @@ def _plan(heads, rows):
         return 0
     units = -(-R // per)
     return -(-units // 16) + heads
+
+
+def _group_plan(groups, rows):
+    """The documented plan of the group-by-group attention: 148 CTAs of 8 warps;
+    per = ceil(R / (148 * 8)) but at least 16, rounded up to a multiple of 16.
+    When per >= rows every range is a whole number of groups (no workspace);
+    otherwise CTA c and group h share slot c + h, 8 heads of 132 floats."""
+    R = groups * rows
+    per = max(-(-R // (148 * 8)), 16)
+    per = (per + 15) // 16 * 16
+    if per >= rows:
+        return 0
+    units = -(-R // per)
+    return -(-units // 8) + groups
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,k", [(1, 32, 8, 131072, 8192), (16, 64, 8, 16384, 1024),
+                                          (2, 8, 2, 1000, 37), (1, 16, 2, 300000, 300000),
+                                          (64, 64, 8, 4096, 256), (3, 12, 4, 16, 16),
+                                          (1, 8, 1, 5000, 5000)])
+def test_group_work_plan_follows_the_documented_rule(B, Hq, Hkv, T, k):
+    """Dense decode and group-shared sparse decode with 2..8 query heads per KV
+    head take the group plan; 1 or more than 8 take the per-head plan."""
+    lib = ds.lib()
+    d = _dims(B=B, Hq=Hq, Hkv=Hkv, T_cap=T, r=8)
+    for op, rows in ((ds.OP_GROUP_SPARSE_DECODE, k), (ds.OP_DECODE, T)):
+        slots = _group_plan(B * Hkv, rows)
+        want = 0 if slots == 0 else (256 * 1024 + slots * 8 * 132 * 4 + 255) // 256 * 256
+        assert lib.ds_workspace_size(op, d, T, k if op == ds.OP_GROUP_SPARSE_DECODE else T) == \
+            want, (op, slots)
+    d16 = _dims(B=B, Hq=16 * Hkv, Hkv=Hkv, T_cap=T, r=8)
+    slots = _plan(B * 16 * Hkv, T)
+    want = 0 if slots == 0 else (256 * 1024 + slots * 132 * 4 + 255) // 256 * 256
+    assert lib.ds_workspace_size(ds.OP_DECODE, d16, T, T) == want
 
 
 @pytest.mark.parametrize("B,H,T,k", [(1, 32, 262144, 16384), (32, 32, 32768, 512),
