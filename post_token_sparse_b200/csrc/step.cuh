@@ -14,14 +14,20 @@
 //               and V rows (K_new, V_new), they are also stored into the K and V
 //               caches here, and the label channels and token T-1's attention
 //               rows are read from K_new / V_new
-//   2. select   the top-k body of topk.cuh; the k indices land in shared memory
-//               (and in idx when requested)
+//   2. select   heads of at most kStepWholeT tokens: every key in shared
+//               memory, then an exact radix select (12-bit histogram of all
+//               keys, 12- and 8-bit histograms of the boundary bin's keys) and
+//               one block scan that places the kept tokens and ranks the ties
+//               (select_whole below); longer heads: the top-k body of
+//               topk.cuh.  The k indices land in shared memory (and in idx
+//               when requested)
 //   3. attend   8 warps each take a contiguous run of the kept rows through a
 //               per-warp cp.async ring (as k_attend does), online softmax in the
 //               log2 domain, warp then CTA merge -> O and lse.
 #pragma once
 
 #include "attend.cuh"
+#include "select.cuh"
 #include "topk.cuh"
 
 namespace ds {
@@ -31,6 +37,11 @@ static_assert(kTopkThreads >= kHeadDim + 48,
               "threads d..d+31 store the new K and V rows, d+32..d+47 load the query row");
 constexpr int kStepStages = 3;
 constexpr int kStepMaxK = 8192;
+constexpr int kStepWholeT = 4096;  // heads selected by select_whole: 16 tokens a thread
+constexpr int kStepTokPerThread = kStepWholeT / kTopkThreads;
+static_assert(kTopkThreads == kSelThreads, "select_whole uses the selector's block scan");
+// shared memory of select_whole, in words: keys, histogram, scan scratch, results
+constexpr int kWholeWords = kStepWholeT + 4096 + 16 + 16;
 
 struct StepParams {
   const uint16_t* Q;
@@ -74,7 +85,9 @@ struct PrefetchSureRows {
 struct StepLayout {
   int over, q, idx, words;
   __host__ __device__ StepLayout(int chunk, int k) {
-    const int sel = TopkLayout(chunk, 1).words;
+    int sel = TopkLayout(chunk, 1).words;
+    const int whole = TopkLayout(chunk, 1).small + 192 + kWholeWords;  // after q at the
+    if (sel < whole) sel = whole;                                         // label channels
     const int att = kStepWarps * kStepStages * kAttnStageU4 * 4 + kStepWarps * 132;
     int o = sel > att ? sel : att;
     o = (o + 3) & ~3;
@@ -89,12 +102,46 @@ struct StepLayout {
   __host__ __device__ size_t bytes() const { return (size_t)words * 4; }
 };
 
+// The threads that run a phase (here the whole CTA): tid() is the index in the
+// group, sync() a barrier over the group.
+struct WholeCta {
+  __device__ __forceinline__ int tid() const { return threadIdx.x; }
+  __device__ __forceinline__ void sync() const { __syncthreads(); }
+};
+
+// Inclusive prefix over a group of kTopkThreads threads, in order; *total: the
+// sum.  scratch: 8 words, not rewritten before the group's next barrier.
+template <class Grp>
+__device__ __forceinline__ uint32_t grp_scan(const Grp& gr, uint32_t v, uint32_t* scratch,
+                                             uint32_t* total) {
+  const int t = gr.tid(), lane = t & 31, w = t >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) scratch[w] = incl;
+  gr.sync();
+  uint32_t base = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < kTopkThreads / 32; ++i) {
+    const uint32_t x = scratch[i];
+    if (i < w) base += x;
+    tot += x;
+  }
+  *total = tot;
+  return base + incl;
+}
+
 // Attention of one query (head bh) over rows idx_s[0..n) of K and V (KV head
-// bkv), by kStepWarps warps; writes O[bh] and lse[bh].
+// bkv), by the kStepWarps warps of group gr; writes O[bh] and lse[bh].
+template <class Grp = WholeCta, int kStages = kStepStages>
 __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv,
                                             const int32_t* idx_s, int n, uint4* ring,
-                                            float* red, const uint4* qrow) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                            float* red, const uint4* qrow,
+                                            const Grp& gr = Grp()) {
+  const int warp = gr.tid() >> 5, lane = gr.tid() & 31;
   const int g = lane >> 3, c = lane & 7;
   float q[16];
   {
@@ -113,7 +160,7 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
   const size_t kv_base = (size_t)bkv * p.T_cap * kHeadDim;
   const uint16_t* Kh = p.K + kv_base;
   const uint16_t* Vh = p.V + kv_base;
-  uint4* my_ring = ring + warp * kStepStages * kAttnStageU4;
+  uint4* my_ring = ring + warp * kStages * kAttnStageU4;
 
   // with K_new, token T-1's rows are read from there: another CTA of the KV
   // group may not have stored them into the caches yet
@@ -127,7 +174,7 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
       const bool nw = Knew != nullptr && t == p.T - 1;
       const uint4* krow = reinterpret_cast<const uint4*>(nw ? Knew : Kh + (size_t)t * kHeadDim);
       const uint4* vrow = reinterpret_cast<const uint4*>(nw ? Vnew : Vh + (size_t)t * kHeadDim);
-      uint4* st = my_ring + (step % kStepStages) * kAttnStageU4 + g * 32;
+      uint4* st = my_ring + (step % kStages) * kAttnStageU4 + g * 32;
       cp_async16(st + c, krow + c);
       cp_async16(st + 8 + c, krow + 8 + c);
       cp_async16(st + 16 + c, vrow + c);
@@ -135,7 +182,7 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
     }
   };
 #pragma unroll
-  for (int s = 0; s < kStepStages - 1; ++s) {
+  for (int s = 0; s < kStages - 1; ++s) {
     if (s < nsteps) issue(s);
     cp_async_commit();
   }
@@ -144,10 +191,10 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   for (int s = 0; s < nsteps; ++s) {
-    if (s + kStepStages - 1 < nsteps) issue(s + kStepStages - 1);
+    if (s + kStages - 1 < nsteps) issue(s + kStages - 1);
     cp_async_commit();
-    cp_async_wait<kStepStages - 1>();
-    const uint4* st = my_ring + (s % kStepStages) * kAttnStageU4 + g * 32;
+    cp_async_wait<kStages - 1>();
+    const uint4* st = my_ring + (s % kStages) * kAttnStageU4 + g * 32;
     const uint4 klo = st[c], khi = st[8 + c];
     float x = dot8(klo, q) + dot8(khi, q + 8);
     x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -182,9 +229,9 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
       wr[1] = l;
     }
   }
-  __syncthreads();
-  if (threadIdx.x < kHeadDim) {
-    const int j = threadIdx.x;
+  gr.sync();
+  if (gr.tid() < kHeadDim) {
+    const int j = gr.tid();
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kStepWarps; ++w) M = fmaxf(M, red[w * 132]);
@@ -197,6 +244,115 @@ __device__ __forceinline__ void attend_rows(const StepParams& p, int bh, int bkv
     }
     p.O[(size_t)bh * kHeadDim + j] = o / L;
     if (p.lse && j == 0) p.lse[bh] = (M + log2f(L)) * 0.69314718055994530942f;
+  }
+}
+
+// In a histogram of nb (256 * q, q a multiple of 4 or 1) bins counted from the
+// top, the bin b holding rank r (1 = largest): res[0] = b, res[1] = count
+// above b.  Ends with a barrier.
+template <class Grp>
+__device__ __forceinline__ void whole_find_bin(const Grp& gr, const uint32_t* hist, int nb,
+                                               uint32_t r, uint32_t* scan, uint32_t* res) {
+  const int q = nb / kTopkThreads;
+  const int lo = nb - (gr.tid() + 1) * q;  // this thread's bins lo .. lo+q-1
+  uint32_t sum = 0;
+#pragma unroll 1
+  for (int i = 0; i < q; i += 4) {
+    if (q >= 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(hist + lo + i);
+      sum += v.x + v.y + v.z + v.w;
+    } else {
+      sum += hist[lo + i];
+    }
+  }
+  uint32_t tot;
+  const uint32_t incl = grp_scan(gr, sum, scan, &tot);
+  uint32_t before = incl - sum;
+  if (before < r && r <= incl) {
+#pragma unroll 1
+    for (int i = q - 1; i >= 0; --i) {
+      const uint32_t c = hist[lo + i];
+      if (before + c >= r) {
+        res[0] = (uint32_t)(lo + i);
+        res[1] = before;
+        break;
+      }
+      before += c;
+    }
+  }
+  gr.sync();
+}
+
+// Top-k of a head of T <= kStepWholeT tokens whose keys are keys[0..T) in
+// shared memory: the k largest, ties to the lower token index, ascending into
+// dst_s (shared) and dst_g (global, may be null).  Exact: the threshold key is
+// fixed digit by digit (bits 31..20 over every key, 19..8 and 7..0 over the
+// keys that share the digits above), then every key above it is kept with the
+// first ties in token order.  The loops are kept rolled: each CTA runs this
+// code once, so its size (instruction fetch) matters more than loop overhead.
+template <class Grp>
+__device__ __noinline__ void select_whole(const Grp gr, const uint32_t* keys, uint32_t* w, int T,
+                                          int k, int32_t* dst_s, int32_t* dst_g) {
+  uint32_t* hist = w;             // 4096 bins
+  uint32_t* scan = w + 4096;      // 16 words
+  uint32_t* res = w + 4096 + 16;  // 16 words
+  uint32_t r = (uint32_t)k, pf = 0u;
+  // digits: (shift, bits) = (20, 12), (8, 12), (0, 8); keys with the prefix pf
+  // above the digit are counted
+#pragma unroll 1
+  for (int d = 0; d < 3; ++d) {
+    const int sh = d == 0 ? 20 : d == 1 ? 8 : 0;
+    const int nb = d == 2 ? 256 : 4096;
+    const int hs = d == 0 ? 32 : d == 1 ? 20 : 8;  // bits above the digit
+#pragma unroll 1
+    for (int i = gr.tid(); i < nb; i += kTopkThreads) hist[i] = 0u;
+    gr.sync();
+#pragma unroll 1
+    for (int t = gr.tid(); t < T; t += kTopkThreads) {
+      const uint32_t key = keys[t];
+      if (hs >= 32 || (key >> hs) == pf) atomicAdd(&hist[(key >> sh) & (uint32_t)(nb - 1)], 1u);
+    }
+    gr.sync();
+    whole_find_bin(gr, hist, nb, r, scan + 8 * (d & 1), res);
+    pf = (pf << (d == 2 ? 8 : 12)) | res[0];
+    r -= res[1];
+    gr.sync();
+  }
+  const uint32_t thr = pf, need_eq = r;  // the k-th key; ties with it kept: need_eq >= 1
+  // this thread's tokens t0 .. t0+15: keys above thr and equal to it
+  const int t0 = gr.tid() * kStepTokPerThread;
+  uint32_t gt = 0u, eq = 0u;
+#pragma unroll 1
+  for (int i = 0; i < kStepTokPerThread; i += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(keys + t0 + i);
+    const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool ok = t0 + i + u < T;
+      gt |= (uint32_t)(ok && kv[u] > thr) << (i + u);
+      eq |= (uint32_t)(ok && kv[u] == thr) << (i + u);
+    }
+  }
+  const uint32_t ngt = __popc(gt), neq = __popc(eq);
+  uint32_t tot;
+  const uint32_t packed = ngt | (neq << 16);
+  const uint32_t excl = grp_scan(gr, packed, scan, &tot) - packed;
+  const uint32_t gt_before = excl & 0xffffu, eq_before = excl >> 16;
+  // the first need_eq ties in token order are kept
+  uint32_t keep = gt, rank = eq_before, m = eq;
+  while (m) {
+    const int i = __ffs(m) - 1;
+    m &= m - 1u;
+    if (rank < need_eq) keep |= 1u << i;
+    ++rank;
+  }
+  uint32_t pos = gt_before + min(eq_before, need_eq);
+  while (keep) {
+    const int i = __ffs(keep) - 1;
+    keep &= keep - 1u;
+    dst_s[pos] = t0 + i;
+    if (dst_g) dst_g[pos] = t0 + i;
+    ++pos;
   }
 }
 
@@ -259,10 +415,26 @@ k_step(const StepParams p, int chunk) {
     src.over_t = p.T - 1;
     src.over_row = reinterpret_cast<const uint4*>(over16);
   }
+  int32_t* dst_g = p.idx ? p.idx + (size_t)bh * p.k : nullptr;
   const size_t kv = (size_t)bkv * p.T_cap * kHeadDim;
   const PrefetchSureRows pf{p.prefetch ? p.K + kv : nullptr, p.V + kv};
-  topk_body(src, sm, 1, 0, bh, p.T, p.k, chunk, p.idx ? p.idx + (size_t)bh * p.k : nullptr,
-            idx_s, true, pf);
+  if (p.T <= kStepWholeT) {
+    // every key into shared memory (the first barrier inside publishes qs and
+    // the new row), then the exact select
+    // keys and the select's scratch after q at the label channels (qs)
+    uint32_t* keys = sm + TopkLayout(chunk, 1).small + 192;
+    for (int i = p.T + threadIdx.x; i < kStepWholeT; i += kTopkThreads) keys[i] = 0u;
+    __syncthreads();
+    src.stream(bh, p.T, p.T, [](int j) { return j; },
+               [&](bool v, int j, uint32_t key, float) {
+                 if (v) keys[j] = key;
+               },
+               qs);
+    __syncthreads();
+    select_whole(WholeCta(), keys, keys + kStepWholeT, p.T, p.k, idx_s, dst_g);
+  } else {
+    topk_body(src, sm, 1, 0, bh, p.T, p.k, chunk, dst_g, idx_s, true, pf);
+  }
   __syncthreads();
 
   // 3. attention over the kept rows (the selection's shared memory is free now)

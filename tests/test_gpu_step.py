@@ -174,3 +174,38 @@ def test_decode_step_kv_equals_kv_append_then_step(case, host):
     L = lse2.cpu().numpy()
     assert np.all(np.abs(L - ref_L) <= 1e-3 * (1 + np.abs(ref_L)))
     assert ds.device_status() == 0
+
+
+@pytest.mark.parametrize("T,k,mode", [(4096, 256, "ints"), (4096, 4096, "ints"), (3000, 2999, "ints"),
+                                      (37, 5, "ints"), (4096, 1000, "zero_q"), (1, 1, "zero_q"),
+                                      (2049, 700, "ints")])
+def test_decode_step_whole_head_ties(T, k, mode):
+    """Heads of at most 4096 tokens are selected in the step kernel from keys held
+    in shared memory.  Scores with many ties (a query of ones over labels in
+    {-1, 0, 1}: integer scores; or a zero query: every score 0) must give the
+    same index set as ds_score_topk and as the oracle's rule (ties to the lower
+    index) applied to the scores ds_score returns."""
+    B, Hq, r = 2, 4, 16
+    w = dsgen.Workload("ties", B=B, Hq=Hq, Hkv=Hq, T=T, r=r, k=k, n_out=8, seed=0x71E + T)
+    inp = gu.Inputs(w, r=r)
+    rng = np.random.default_rng(T + k)
+    lab = rng.integers(-1, 2, size=(B, Hq, T, r)).astype(np.float32)
+    label = torch.from_numpy(lab).to(torch.bfloat16).cuda()
+    Q = torch.zeros_like(inp.dQ) if mode == "zero_q" else torch.ones_like(inp.dQ)
+    idx = torch.full((B * Hq, k), -1, dtype=torch.int32, device="cuda")
+    O = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+    ds.decode_step(Q, inp.dK, inp.dV, inp.dC, label, idx, O, T, w.scale, append=False)
+    idx_sep = torch.empty_like(idx)
+    ds.score_topk(Q, inp.dC, label, idx_sep, T)
+    s = torch.empty((B * Hq, T), dtype=torch.float32, device="cuda")
+    ds.score(Q, inp.dC, label, s, T)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_sep)
+    S = s.cpu().numpy()
+    I = idx.cpu().numpy()
+    for bh in range(B * Hq):
+        assert np.array_equal(I[bh], oracle.topk_head(S[bh], k)), bh
+    if mode == "zero_q":
+        assert np.array_equal(I, np.tile(np.arange(k, dtype=np.int32), (B * Hq, 1)))
+    assert ds.device_status() == 0
+    inp.free()
