@@ -305,10 +305,8 @@ ds_status ds_decode(const void* Q, const void* K, const void* V, float* O, float
  * DS_ERR_UNSUPPORTED.
  *
  * The first call on each device looks up the array's device address with
- * that device current (cudaGetSymbolAddress); make that first call outside
- * any stream capture: until the address is known, a call on a stream that is
- * being captured returns DS_ERR_UNSUPPORTED and launches nothing.  All calls
- * on a device share the one array and it keeps the previous call's contents.
+ * that device current (cudaGetSymbolAddress).  All calls on a device share
+ * the one array and it keeps the previous call's contents.
  * Its layout is that of the ds_sparse_decode workspace: the per-head counters
  * sit at its start, are zero when the library is loaded and are left at zero
  * by every call, so no call has to clear anything first.  Calls that may

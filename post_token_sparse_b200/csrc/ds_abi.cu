@@ -694,19 +694,14 @@ cudaError_t g_scratch_err[kMaxDevices];
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name is only a host-side handle, so the address is looked up once
-// per device, with that device current.  The lookup is refused while `stream`
-// is being captured into a graph (the first call must come before capture).
-ds_status noalloc_scratch(cudaStream_t stream, void** out) {
+// per device, with that device current.
+ds_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return DS_ERR_UNSUPPORTED;
   void* a = g_scratch_addr[dev].load(std::memory_order_acquire);
   if (a == nullptr) {
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    e = cudaStreamIsCapturing(stream, &cap);
-    if (e != cudaSuccess) return cuda_fail(e);
-    if (cap != cudaStreamCaptureStatusNone) return DS_ERR_UNSUPPORTED;
     std::call_once(g_scratch_once[dev], [dev] {
       void* p = nullptr;
       g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
@@ -739,7 +734,7 @@ extern "C" ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, cons
   if (s != DS_OK) return s;
   void* scratch = nullptr;
   if (need > 0) {
-    s = noalloc_scratch(stream, &scratch);
+    s = noalloc_scratch(&scratch);
     if (s != DS_OK) return s;
   }
   return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, scratch, stream);
