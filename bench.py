@@ -668,11 +668,10 @@ def group_entry(w, inputs, hbm_peak, steps: int = 50):
     idx = torch.empty((w.B * w.Hkv, w.k), dtype=torch.int32, device="cuda")
     O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
     ws = ds.workspace(ds.OP_GROUP_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
-    ws_sel = ds.workspace(ds.OP_GROUP_SCORE_TOPK, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
 
     def step():
         ds.label_append(K, C, label, w.T - 1, 1)
-        ds.group_score_topk(Q, C, label, sg, idx, w.T, ws=ws_sel)
+        ds.group_score_topk(Q, C, label, sg, idx, w.T)
         ds.group_sparse_decode(Q, K, V, idx, O, w.T, w.scale, ws=ws)
 
     ms = time_graph(step, steps, 3)

@@ -92,8 +92,7 @@ enum {
   DS_OP_DECODE_STEP = 6,
   DS_OP_CALIBRATE = 7, /* k: calibration queries per head (Nq) */
   DS_OP_GROUP_SPARSE_DECODE = 8,
-  DS_OP_BLOCK_SPARSE_DECODE = 9, /* k: kept rows = kb * bs */
-  DS_OP_GROUP_SCORE_TOPK = 10
+  DS_OP_BLOCK_SPARSE_DECODE = 9 /* k: kept rows = kb * bs */
 };
 
 /* Device status bits (ds_device_status). */
@@ -333,18 +332,11 @@ ds_status ds_sparse_decode_noalloc(const void* Q, const void* K, const void* V,
  * Q: [B,Hq,d] bf16.  C: [Hq,r] int32.  label: [B,Hq,T_cap,r] bf16.
  * group_scores: [B*Hkv, T] fp32 (written; the caller's buffer).  idx:
  * [B*Hkv, k] int32.  Requires r in {8,16,32,64,128}, G*r <= 12288,
- * 1 <= k <= T <= min(T_cap, 1048576).
- * ws: NULL, or ds_workspace_size(DS_OP_GROUP_SCORE_TOPK, dims, T, k) bytes of
- * 16-byte aligned device memory, zero-filled before its first use (its
- * counters are left at zero).  When that size is nonzero (4096 < T <= 32768
- * and G*r <= 1024) and ws is given, one launch computes the group scores in
- * tiles of 2048 tokens and the last tile of each group selects from 16-bit
- * key prefixes kept in ws; otherwise two launches (group scores, then the
- * top-k over them).  Same result either way.
+ * 1 <= k <= T <= min(T_cap, 1048576).  Two launches.
  */
 ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
                               float* group_scores, int32_t* idx, ds_dims dims, int32_t T,
-                              int32_t k, void* ws, size_t ws_bytes, ds_stream_t stream);
+                              int32_t k, ds_stream_t stream);
 
 /*
  * ds_group_sparse_decode -- attention over the group's kept tokens.

@@ -33,8 +33,7 @@ LIB_PATH = os.path.join(_HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
 (OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK,
- OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE,
- OP_GROUP_SCORE_TOPK) = range(11)
+ OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE) = range(10)
 DEV_BAD_CHANNEL, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
 
 
@@ -77,7 +76,7 @@ def _load():
         "ds_decode_step_kv": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32,
                               ctypes.c_float, vp, ctypes.c_size_t, vp],
         "ds_calibrate": [vp, i32, vp, Dims, i32, vp, vp, vp, ctypes.c_size_t, vp],
-        "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp, ctypes.c_size_t, vp],
+        "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
         "ds_hier_score_topk": [vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_kv_append": [vp, vp, vp, vp, Dims, i32, vp],
@@ -284,22 +283,16 @@ def decode(Q, K, V, O, T: int, scale: float, lse=None, ws=None):
                           _ptr(ws, None, "ws"), nbytes, _stream(Q.device)), "ds_decode")
 
 
-def group_score_topk(Q, C, label, group_scores, idx, T: int, ws=None):
-    """One selection per KV group: group_scores [B*Hkv, T] fp32, idx [B*Hkv, k]; ws:
-    the workspace of OP_GROUP_SCORE_TOPK (made here when not given)."""
+def group_score_topk(Q, C, label, group_scores, idx, T: int):
+    """One selection per KV group: group_scores [B*Hkv, T] fp32, idx [B*Hkv, k]."""
     B, Hq, T_cap, r = label.shape
     Hkv = group_scores.shape[0] // B
     dims = Dims(B, Hq, Hkv, Q.shape[-1], T_cap, r)
-    k = idx.shape[-1]
-    if ws is None:
-        ws = workspace(OP_GROUP_SCORE_TOPK, dims, T, k, Q.device)
-    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.ds_group_score_topk(_ptr(Q, torch.bfloat16, "Q"), _ptr(C, torch.int32, "C"),
                                     _ptr(label, torch.bfloat16, "label"),
                                     _ptr(group_scores, torch.float32, "group_scores"),
-                                    _ptr(idx, torch.int32, "idx"), dims, T, k,
-                                    _ptr(ws, None, "ws"), nbytes, _stream(Q.device)),
-           "ds_group_score_topk")
+                                    _ptr(idx, torch.int32, "idx"), dims, T, idx.shape[-1],
+                                    _stream(Q.device)), "ds_group_score_topk")
 
 
 def group_sparse_decode(Q, K, V, idx, O, T: int, scale: float, lse=None, ws=None):

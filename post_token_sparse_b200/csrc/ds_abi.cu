@@ -295,33 +295,6 @@ ds_status launch_sel(const uint16_t* Q, const int32_t* C, const uint16_t* label,
   return launched();
 }
 
-// One-launch group selection: as sel_applies, with the group's query values
-// (G * r floats) in the CTA's shared memory.
-bool grp_sel_applies(const ds_dims& d, int T) {
-  return sel_applies(d.r, T) && (d.Hq / d.Hkv) * d.r <= kGrpSelMaxQ;
-}
-
-template <int R>
-ds_status launch_grp_sel(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* sg,
-                         int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
-  SelParams sp;
-  sp.Q = Q;
-  sp.C = C;
-  sp.label = label;
-  sp.scores = sg;
-  sp.idx = idx;
-  sp.arrivals = static_cast<uint32_t*>(ws);
-  sp.prefixes = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kCounterBytes);
-  sp.BH = d.B * d.Hkv;
-  sp.Hq = d.Hq;
-  sp.T_cap = d.T_cap;
-  sp.T = T;
-  sp.k = k;
-  dim3 grid((T + kGrpSelTile - 1) / kGrpSelTile, sp.BH);
-  k_group_score_select<R><<<grid, kSelThreads, 0, st>>>(sp, d.Hkv);
-  return launched();
-}
-
 ds_status score_select(const uint16_t* Q, const int32_t* C, const uint16_t* label, float* scores,
                        int32_t* idx, const ds_dims& d, int T, int k, void* ws, cudaStream_t st) {
   switch (d.r) {
@@ -519,9 +492,6 @@ size_t ds_workspace_size(int32_t op, ds_dims dims, int32_t T, int32_t k) {
     case DS_OP_GROUP_SPARSE_DECODE:
       if (k < 1 || k > T) return 0;
       return shared_rows_ws_bytes(dims, k);
-    case DS_OP_GROUP_SCORE_TOPK:
-      if (k < 1 || k > T) return 0;
-      return grp_sel_applies(dims, T) ? sel_ws_bytes(dims.B * dims.Hkv, T) : 0;
     case DS_OP_CALIBRATE: {
       if (k < 1) return 0;  // k: calibration queries per head
       const size_t nck = (T + kAbsumRows - 1) / kAbsumRows, ncq = (k + kAbsumRows - 1) / kAbsumRows;
@@ -901,8 +871,7 @@ ds_status launch_group_score(const uint16_t* Q, const int32_t* C, const uint16_t
 
 extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const void* label,
                                          float* group_scores, int32_t* idx, ds_dims dims,
-                                         int32_t T, int32_t k, void* ws, size_t ws_bytes,
-                                         ds_stream_t stream) {
+                                         int32_t T, int32_t k, ds_stream_t stream) {
   DS_TRACE("ds_group_score_topk");
   ds_status s = check_dims(dims);
   if (s != DS_OK) return s;
@@ -919,16 +888,6 @@ extern "C" ds_status ds_group_score_topk(const void* Q, const int32_t* C, const 
   if (s != DS_OK) return s;
   auto Qb = static_cast<const uint16_t*>(Q);
   auto Lb = static_cast<const uint16_t*>(label);
-  if (grp_sel_applies(dims, T) && ws && aligned16(ws) &&
-      ws_bytes >= sel_ws_bytes(dims.B * dims.Hkv, T)) {
-    switch (dims.r) {
-      case 8: return launch_grp_sel<8>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
-      case 16: return launch_grp_sel<16>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
-      case 32: return launch_grp_sel<32>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
-      case 64: return launch_grp_sel<64>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
-      default: return launch_grp_sel<128>(Qb, C, Lb, group_scores, idx, dims, T, k, ws, stream);
-    }
-  }
   switch (dims.r) {
     case 8: s = launch_group_score<8>(Qb, C, Lb, group_scores, dims, T, stream); break;
     case 16: s = launch_group_score<16>(Qb, C, Lb, group_scores, dims, T, stream); break;

@@ -128,9 +128,8 @@ __device__ __forceinline__ void exact_keys(const uint16_t* lab, const float* qs,
   }
 }
 
-// Exact keys of a head's tokens for the selection's boundary bin: recomputed
-// from the head's label rows (LabelKeys), or read from the scores the tile
-// CTAs wrote (StoredKeys: written by other CTAs of the launch, read around L1).
+// Exact keys of a head's tokens for the selection's boundary bin, recomputed
+// from the head's label rows.
 template <int R>
 struct LabelKeys {
   const uint16_t* lab;
@@ -142,27 +141,6 @@ struct LabelKeys {
     exact_keys<R>(lab, qs, tok, key, n);
   }
 };
-struct StoredKeys {
-  const float* sc;
-  __device__ __forceinline__ uint32_t key(int t) const { return order_key(__ldcg(sc + t)); }
-  __device__ __forceinline__ void keys(const uint32_t* tok, uint32_t* key, int n) const {
-    constexpr int kB = 4;
-    for (int i0 = threadIdx.x; i0 < n; i0 += kB * kSelThreads) {
-      float v[kB];
-#pragma unroll
-      for (int j = 0; j < kB; ++j) {
-        const int i = i0 + j * kSelThreads;
-        v[j] = i < n ? __ldcg(sc + tok[i]) : 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < kB; ++j) {
-        const int i = i0 + j * kSelThreads;
-        if (i < n) key[i] = order_key(v[j]);
-      }
-    }
-  }
-};
-
 // Inclusive prefix over the CTA's threads in order; *total: the sum.
 // scratch: 8 words, not rewritten before the caller's next barrier.
 __device__ __forceinline__ uint32_t blk_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
@@ -542,93 +520,6 @@ k_score_select(const SelParams p) {
   __threadfence();
   select_head(p, bh, s, LabelKeys<R>{p.label + (size_t)bh * p.T_cap * R, s.qs});
   if (threadIdx.x == 0) p.arrivals[bh] = 0u;  // zero again for the next call
-}
-
-// ---- group-shared selection in one launch -------------------------------------
-//
-// Grouped KV heads with one selection per KV group (group score: the sum of
-// the member heads' scores, in head order, as k_group_score computes it).
-// Grid (ceil(T / kGrpSelTile), B*Hkv): each CTA streams the label rows of the
-// G heads for one tile of tokens, writes the group scores (an output) and the
-// 16-bit key prefixes, and the group's last tile selects exactly as above,
-// taking the boundary bin's exact keys from the group scores just written.
-constexpr int kGrpSelTile = 2048;  // tokens per CTA: G label rows each
-constexpr int kGrpSelMaxQ = 1024;  // G * r floats of query values in shared memory
-
-template <int R>
-__global__ void __launch_bounds__(kSelThreads, 3)
-k_group_score_select(const SelParams p, int Hkv) {
-  using S = ScoreShape<R>;
-  __shared__ SelSmem s;
-  __shared__ __align__(16) float qg[kGrpSelMaxQ];  // [G][R]
-  const int Hq = p.Hq, G = Hq / Hkv;
-  const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
-  for (int i = threadIdx.x; i < G * R; i += kSelThreads) {
-    const int hh = i / R, j = i % R;
-    const int h = g * G + hh;
-    int c = p.C[h * R + j];
-    if (c < 0 || c >= kHeadDim) {
-      flag_status(1u);
-      c &= (kHeadDim - 1);
-    }
-    qg[i] = bf_at(p.Q + (size_t)(b * Hq + h) * kHeadDim + c);
-  }
-  __syncthreads();
-  const int T = p.T, per = sel_per(T);
-  uint16_t* pref = p.prefixes + (size_t)bg * per * kSelThreads;
-  float* so = p.scores + (size_t)bg * T;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int chunk = lane % S::kLanes;
-  const int t_end = min(T, (int)(blockIdx.x + 1) * kGrpSelTile);
-  for (int base = blockIdx.x * kGrpSelTile; base < t_end; base += S::kTokensPerCta) {
-    auto token = [&](int i) {
-      return base + (warp * S::kSlots + i) * S::kRowsPerInstr + lane / S::kLanes;
-    };
-    float acc[S::kSlots];
-    // two heads' rows loaded before either is used; head order in the sum
-    for (int hh = 0; hh < G; hh += 2) {
-      const bool two = hh + 1 < G;
-      const uint4* lab0 = reinterpret_cast<const uint4*>(
-          p.label + (size_t)(b * Hq + g * G + hh) * p.T_cap * R);
-      const uint4* lab1 = lab0 + (size_t)p.T_cap * S::kLanes;
-      uint4 v0[S::kSlots], v1[S::kSlots];
-#pragma unroll
-      for (int i = 0; i < S::kSlots; ++i) {
-        const int t = token(i);
-        v0[i] = t < t_end ? ldg_stream(lab0 + (size_t)t * S::kLanes + chunk)
-                          : make_uint4(0, 0, 0, 0);
-        v1[i] = two && t < t_end ? ldg_stream(lab1 + (size_t)t * S::kLanes + chunk)
-                                 : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < S::kSlots; ++i) {
-        const float s0 = lane_group_score<R>(v0[i], qg + hh * R, chunk);
-        acc[i] = hh == 0 ? s0 : acc[i] + s0;
-        if (two) {
-          const float s1 = lane_group_score<R>(v1[i], qg + (hh + 1) * R, chunk);
-          acc[i] = acc[i] + s1;
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < S::kSlots; ++i) {
-      const int t = token(i);
-      if (t < t_end && chunk == 0) {
-        so[t] = acc[i];
-        pref[key_slot(t, per)] = (uint16_t)(order_key(acc[i]) >> 16);
-      }
-    }
-  }
-  // the group's last tile to finish selects it
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0)
-    s.misc[S_LAST] = atomicAdd(&p.arrivals[bg], 1u) == gridDim.x - 1 ? 1u : 0u;
-  __syncthreads();
-  if (s.misc[S_LAST] == 0u) return;
-  __threadfence();
-  select_head(p, bg, s, StoredKeys{so});
-  if (threadIdx.x == 0) p.arrivals[bg] = 0u;  // zero again for the next call
 }
 
 }  // namespace ds

@@ -169,29 +169,17 @@ def test_decode_step_fuses_only_one_wave_of_heads():
                                  32768, 2048) > 0
 
 
-def test_group_score_topk_workspace():
-    """One-launch group selection for 4096 < T <= 32768 and G*r <= 1024: the
-    arrival counters, then 16-bit prefixes of every group's padded T."""
-    lib = ds.lib()
-    d = _dims(B=16, Hq=64, Hkv=8, T_cap=16384, r=16)
-    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, d, 16384, 1024) == \
-        256 * 1024 + 128 * 16384 * 2
-    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, d, 4096, 100) == 0
-    assert lib.ds_workspace_size(ds.OP_GROUP_SCORE_TOPK, _dims(B=1, Hq=64, Hkv=4, T_cap=9000,
-                                                               r=128), 9000, 10) == 0
-
-
 def test_group_calls_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG
     d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
     mis = ctypes.c_void_p(FAKE + 4)
-    assert lib.ds_group_score_topk(P, P, P, NUL, P, d, 100, 10, NUL, 0, NUL) == bad  # scores required
-    assert lib.ds_group_score_topk(P, P, P, P, P, d, 100, 101, NUL, 0, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, d, 1001, 10, NUL, 0, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, mis, P, d, 100, 10, NUL, 0, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(Hq=6, Hkv=4), 100, 10, NUL, 0, NUL) == bad
-    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(r=12), 100, 10, NUL, 0, NUL) == \
+    assert lib.ds_group_score_topk(P, P, P, NUL, P, d, 100, 10, NUL) == bad  # scores required
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 100, 101, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, d, 1001, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, mis, P, d, 100, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(Hq=6, Hkv=4), 100, 10, NUL) == bad
+    assert lib.ds_group_score_topk(P, P, P, P, P, _dims(r=12), 100, 10, NUL) == \
         ds.DS_ERR_UNSUPPORTED
     assert lib.ds_group_sparse_decode(P, P, P, P, P, NUL, d, 100, 101, 1.0, NUL, 0, NUL) == bad
     assert lib.ds_group_sparse_decode(P, P, P, NUL, P, NUL, d, 100, 10, 1.0, NUL, 0, NUL) == bad

@@ -30,11 +30,10 @@ CASES = [
     ("g4-r128-ragged", 1, 8, 2, 777, 800, 128, 77),
     ("long-cluster", 1, 4, 1, 40000, 40000, 8, 2500),
     ("k-equals-T", 1, 4, 2, 96, 96, 16, 96),
-    # one launch (4096 < T <= 32768, G*r <= 1024): tiles of 2048 tokens
-    ("fused-g8-r128", 1, 16, 2, 9000, 9000, 128, 500),
-    ("fused-g2-r8-T32768", 1, 4, 2, 32768, 32768, 8, 4000),
-    ("fused-g4-k1-ragged", 2, 8, 2, 4097, 4100, 16, 1),
-    ("fused-g3-kT", 1, 6, 2, 6000, 6000, 16, 6000),
+    ("g8-r128", 1, 16, 2, 9000, 9000, 128, 500),
+    ("g2-r8-T32768", 1, 4, 2, 32768, 32768, 8, 4000),
+    ("g4-k1-ragged", 2, 8, 2, 4097, 4100, 16, 1),
+    ("g3-kT", 1, 6, 2, 6000, 6000, 16, 6000),
 ]
 
 
@@ -125,51 +124,3 @@ def test_group_full_workload_sampled():
             assert np.abs(On[b, h] - o).max() <= 1e-2
     inp.free()
 
-
-def _raw_group_select(Q, C, label, sg, idx, T, Hkv, ws):
-    """ds_group_score_topk through the C ABI with an explicit workspace (None:
-    the two-launch path)."""
-    import ctypes
-    B, Hq, T_cap, r = label.shape
-    dims = ds.Dims(B, Hq, Hkv, Q.shape[-1], T_cap, r)
-    st = ds.lib().ds_group_score_topk(
-        ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(C.data_ptr()),
-        ctypes.c_void_p(label.data_ptr()), ctypes.c_void_p(sg.data_ptr()),
-        ctypes.c_void_p(idx.data_ptr()), dims, T, idx.shape[-1],
-        None if ws is None else ctypes.c_void_p(ws.data_ptr()),
-        0 if ws is None else ws.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    assert st == ds.DS_OK, ds.lib().ds_status_string(st)
-
-
-@pytest.mark.parametrize("B,Hq,Hkv,T,r,k,zero_q", [
-    (2, 16, 2, 16384, 16, 1024, False),
-    (1, 8, 1, 20000, 32, 3000, False),
-    (1, 8, 2, 12000, 8, 700, True),    # every group score 0: ties to the lower index
-])
-def test_group_one_launch_equals_two_launches(B, Hq, Hkv, T, r, k, zero_q):
-    w = dsgen.Workload("g-fused", B=B, Hq=Hq, Hkv=Hkv, T=T, r=r, k=k, n_out=min(16, r),
-                       seed=0x6F0 + T)
-    inp = gu.Inputs(w, r=r)
-    Q = torch.zeros_like(inp.dQ) if zero_q else inp.dQ
-    label = torch.empty((B, Hq, T, r), dtype=torch.bfloat16, device="cuda")
-    ds.label_append(inp.dK, inp.dC, label, 0, T)
-    dims = ds.Dims(B, Hq, Hkv, 128, T, r)
-    ws = ds.workspace(ds.OP_GROUP_SCORE_TOPK, dims, T, k, "cuda")
-    assert ws is not None
-    sg1 = torch.full((B * Hkv, T), float("nan"), dtype=torch.float32, device="cuda")
-    sg2 = torch.full_like(sg1, float("nan"))
-    i1 = torch.full((B * Hkv, k), -1, dtype=torch.int32, device="cuda")
-    i2 = torch.full_like(i1, -1)
-    for rep in range(2):  # the workspace is reused: its counters are left at zero
-        _raw_group_select(Q, inp.dC, label, sg1, i1, T, Hkv, ws)
-        _raw_group_select(Q, inp.dC, label, sg2, i2, T, Hkv, None)
-        torch.cuda.synchronize()
-        assert torch.equal(sg1, sg2)
-        assert torch.equal(i1, i2)
-    assert int(ws.view(torch.int32)[: B * Hkv].abs().sum()) == 0
-    SG = sg1.cpu().numpy().reshape(B, Hkv, T)
-    assert np.array_equal(i1.cpu().numpy().reshape(B, Hkv, k), oracle.topk(SG, k))
-    if zero_q:
-        assert np.array_equal(i1.cpu().numpy(), np.tile(np.arange(k, dtype=np.int32), (B * Hkv, 1)))
-    assert ds.device_status() == 0
-    inp.free()
