@@ -653,9 +653,9 @@ def calib_entry(w, K, hbm_peak, nq: int = 16, steps: int = 50):
 
 
 def group_entry(w, inputs, hbm_peak, steps: int = 50):
-    """Group-shared selection on grouped KV heads: the step's label append,
-    ds_group_score_topk and ds_group_sparse_decode (one selection per KV group,
-    each kept row read once for the group's query heads)."""
+    """Group-shared selection on grouped KV heads: ds_group_decode_step (the step's
+    label append, group scores, one selection per KV group, attention with each kept
+    row read once for the group's query heads; three launches)."""
     import torch
 
     import post_token_sparse_b200 as ds
@@ -670,9 +670,7 @@ def group_entry(w, inputs, hbm_peak, steps: int = 50):
     ws = ds.workspace(ds.OP_GROUP_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
 
     def step():
-        ds.label_append(K, C, label, w.T - 1, 1)
-        ds.group_score_topk(Q, C, label, sg, idx, w.T)
-        ds.group_sparse_decode(Q, K, V, idx, O, w.T, w.scale, ws=ws)
+        ds.group_decode_step(Q, K, V, C, label, sg, idx, O, w.T, w.scale, ws=ws)
 
     ms = time_graph(step, steps, 3)
     nb = w.group_step_bytes()

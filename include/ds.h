@@ -354,6 +354,24 @@ ds_status ds_group_sparse_decode(const void* Q, const void* K, const void* V,
                                  ds_stream_t stream);
 
 /*
+ * ds_group_decode_step -- one decode step with group-shared selection:
+ * ds_label_append(K, C, label, dims, T-1, 1) (when append != 0), then
+ * ds_group_score_topk and ds_group_sparse_decode, in three launches instead
+ * of four: the group-score kernel appends the newest token's label rows (the
+ * CTA whose tile holds token T-1 gathers them from K) and scores that token
+ * from them.  Results identical to the three calls.
+ *
+ * Arguments as for those calls (label written at T-1 when append != 0).  ws:
+ * ds_workspace_size(DS_OP_GROUP_SPARSE_DECODE, dims, T, k) bytes, zero-filled
+ * before first use.  Requires what ds_group_score_topk requires, with
+ * G*r*6 <= 49152.
+ */
+ds_status ds_group_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
+                               void* label, float* group_scores, int32_t* idx, float* O,
+                               float* lse, ds_dims dims, int32_t T, int32_t k, float scale,
+                               int32_t append, void* ws, size_t ws_bytes, ds_stream_t stream);
+
+/*
  * ds_block_score_topk -- block-granular token selection.
  *
  * Block informativeness (page "Jenga: Enhancing LLM Long-Context Fine-tuning

@@ -77,6 +77,8 @@ def _load():
                               ctypes.c_float, vp, ctypes.c_size_t, vp],
         "ds_calibrate": [vp, i32, vp, Dims, i32, vp, vp, vp, ctypes.c_size_t, vp],
         "ds_group_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, vp],
+        "ds_group_decode_step": [vp, vp, vp, vp, vp, vp, vp, vp, vp, Dims, i32, i32,
+                                 ctypes.c_float, i32, vp, ctypes.c_size_t, vp],
         "ds_block_score_topk": [vp, vp, vp, vp, vp, Dims, i32, i32, i32, vp],
         "ds_hier_score_topk": [vp, vp, vp, vp, Dims, i32, i32, vp],
         "ds_kv_append": [vp, vp, vp, vp, Dims, i32, vp],
@@ -293,6 +295,26 @@ def group_score_topk(Q, C, label, group_scores, idx, T: int):
                                     _ptr(group_scores, torch.float32, "group_scores"),
                                     _ptr(idx, torch.int32, "idx"), dims, T, idx.shape[-1],
                                     _stream(Q.device)), "ds_group_score_topk")
+
+
+def group_decode_step(Q, K, V, C, label, group_scores, idx, O, T: int, scale: float,
+                      append: bool = True, lse=None, ws=None):
+    """Label row of token T-1 (if append), group-shared selection and attention, three
+    launches: group_scores [B*Hkv, T], idx [B*Hkv, k], O [B, Hq, d]."""
+    B, Hq, T_cap, r = label.shape
+    Hkv = K.shape[1]
+    dims = Dims(B, Hq, Hkv, Q.shape[-1], T_cap, r)
+    k = idx.shape[-1]
+    if ws is None:
+        ws = workspace(OP_GROUP_SPARSE_DECODE, dims, T, k, Q.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.ds_group_decode_step(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
+        _ptr(C, torch.int32, "C"), _ptr(label, torch.bfloat16, "label"),
+        _ptr(group_scores, torch.float32, "group_scores"), _ptr(idx, torch.int32, "idx"),
+        _ptr(O, torch.float32, "O"), _ptr(lse, torch.float32, "lse"), dims, T, k, scale,
+        int(bool(append)), _ptr(ws, None, "ws"), nbytes, _stream(Q.device)),
+        "ds_group_decode_step")
 
 
 def group_sparse_decode(Q, K, V, idx, O, T: int, scale: float, lse=None, ws=None):

@@ -856,14 +856,17 @@ extern "C" ds_status ds_calibrate(const void* Qc, int32_t Nq, const void* K, ds_
 
 namespace {
 
+// Kc: the K cache when the newest token's label rows are appended first, else null.
 template <int R>
 ds_status launch_group_score(const uint16_t* Q, const int32_t* C, const uint16_t* label,
-                             float* sg, const ds_dims& d, int T, cudaStream_t st) {
+                             float* sg, const ds_dims& d, int T, cudaStream_t st,
+                             const uint16_t* Kc = nullptr) {
   using S = ScoreShape<R>;
   const int G = d.Hq / d.Hkv;
   dim3 grid((T + S::kTokensPerCta - 1) / S::kTokensPerCta, d.B * d.Hkv);
-  k_group_score<R><<<grid, kScoreThreads, (size_t)G * R * sizeof(float), st>>>(
-      Q, C, label, sg, d.Hq, d.Hkv, d.T_cap, T);
+  const size_t smem = (size_t)G * R * (sizeof(float) + (Kc ? 2 : 0));
+  k_group_score<R><<<grid, kScoreThreads, smem, st>>>(Q, C, const_cast<uint16_t*>(label), sg,
+                                                      d.Hq, d.Hkv, d.T_cap, T, Kc);
   return launched();
 }
 
@@ -916,6 +919,48 @@ extern "C" ds_status ds_group_sparse_decode(const void* Q, const void* K, const 
   s = check_kv(K, V);
   if (s != DS_OK) return s;
   s = ensure_attrs();
+  if (s != DS_OK) return s;
+  if (group_kernel_applies(dims))
+    return launch_attend_group(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);
+  return launch_attend(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream, true);
+}
+
+extern "C" ds_status ds_group_decode_step(const void* Q, const void* K, const void* V,
+                                          const int32_t* C, void* label, float* group_scores,
+                                          int32_t* idx, float* O, float* lse, ds_dims dims,
+                                          int32_t T, int32_t k, float scale, int32_t append,
+                                          void* ws, size_t ws_bytes, ds_stream_t stream) {
+  DS_TRACE("ds_group_decode_step");
+  ds_status s = check_dims(dims);
+  if (s != DS_OK) return s;
+  if (!Q || !K || !V || !C || !label || !group_scores || !idx || !O || !aligned16(Q) ||
+      !aligned16(K) || !aligned16(V) || !aligned16(C) || !aligned16(label) ||
+      !aligned16(group_scores) || !aligned16(idx) || !aligned16(O) || (lse && !aligned16(lse)))
+    return DS_ERR_INVALID_ARG;
+  if (T < 1 || T > dims.T_cap || k < 1 || k > T) return DS_ERR_INVALID_ARG;
+  if (T > kMaxCluster * kMaxKeysPerCta) return DS_ERR_UNSUPPORTED;
+  const int G = dims.Hq / dims.Hkv;
+  if ((size_t)G * dims.r * (sizeof(float) + 2) > 48 * 1024) return DS_ERR_UNSUPPORTED;
+  if (!(dims.r == 8 || dims.r == 16 || dims.r == 32 || dims.r == 64 || dims.r == 128))
+    return DS_ERR_UNSUPPORTED;
+  s = check_shared_rows_ws(dims, k, ws, ws_bytes);
+  if (s != DS_OK) return s;
+  s = check_kv(K, V);
+  if (s != DS_OK) return s;
+  s = ensure_attrs();
+  if (s != DS_OK) return s;
+  auto Qb = static_cast<const uint16_t*>(Q);
+  auto Lb = static_cast<const uint16_t*>(label);
+  const uint16_t* Kc = append ? static_cast<const uint16_t*>(K) : nullptr;
+  switch (dims.r) {
+    case 8: s = launch_group_score<8>(Qb, C, Lb, group_scores, dims, T, stream, Kc); break;
+    case 16: s = launch_group_score<16>(Qb, C, Lb, group_scores, dims, T, stream, Kc); break;
+    case 32: s = launch_group_score<32>(Qb, C, Lb, group_scores, dims, T, stream, Kc); break;
+    case 64: s = launch_group_score<64>(Qb, C, Lb, group_scores, dims, T, stream, Kc); break;
+    default: s = launch_group_score<128>(Qb, C, Lb, group_scores, dims, T, stream, Kc); break;
+  }
+  if (s != DS_OK) return s;
+  s = launch_topk(ScoresSource{group_scores}, idx, dims.B * dims.Hkv, T, k, stream);
   if (s != DS_OK) return s;
   if (group_kernel_applies(dims))
     return launch_attend_group(dims, Q, K, V, idx, O, lse, T, k, scale, ws, stream);

@@ -124,16 +124,24 @@ namespace ds {
 // computes it and the sum taken in head order in fp32 (group-shared
 // selection: one top-k per KV group, so that each selected K/V row is read
 // once for all of the group's query heads).
-// grid: (ceil(T / kTokensPerCta), B*Hkv); dynamic shared memory G*R floats.
+// With Kc (the K cache, [B, Hkv, T_cap, d]) the newest token's label rows are
+// appended first, as ds_label_append(.., T-1, 1) writes them: the CTA whose
+// tile holds token T-1 gathers them from K into shared memory and the label
+// cache, and scores that token from shared memory.
+// grid: (ceil(T / kTokensPerCta), B*Hkv); dynamic shared memory G*R floats,
+// then (with Kc) G*R bf16.
 template <int R>
 __global__ void __launch_bounds__(kScoreThreads)
-k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
-              const uint16_t* __restrict__ label, float* __restrict__ sg, int Hq, int Hkv,
-              int T_cap, int T) {
+k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C, uint16_t* label,
+              float* __restrict__ sg, int Hq, int Hkv, int T_cap, int T,
+              const uint16_t* __restrict__ Kc) {
   using S = ScoreShape<R>;
   extern __shared__ __align__(16) float qg[];  // [G][R]
   const int G = Hq / Hkv;
+  uint16_t* newrow = reinterpret_cast<uint16_t*>(qg + G * R);  // [G][R] with Kc
   const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+  const int t_new = T - 1;
+  const bool app = Kc != nullptr && t_new / S::kTokensPerCta == (int)blockIdx.x;
   for (int i = threadIdx.x; i < G * R; i += blockDim.x) {
     const int hh = i / R, j = i % R;
     const int h = g * G + hh;
@@ -143,6 +151,11 @@ k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
       c &= (kHeadDim - 1);
     }
     qg[i] = bf_at(Q + (size_t)(b * Hq + h) * kHeadDim + c);
+    if (app) {
+      const uint16_t v = Kc[((size_t)bg * T_cap + t_new) * kHeadDim + c];
+      newrow[i] = v;
+      label[((size_t)(b * Hq + h) * T_cap + t_new) * R + j] = v;
+    }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -165,6 +178,11 @@ k_group_score(const uint16_t* __restrict__ Q, const int32_t* __restrict__ C,
       v0[i] = t < T ? ldg_stream(lab0 + (size_t)t * S::kLanes + chunk) : make_uint4(0, 0, 0, 0);
       v1[i] = two && t < T ? ldg_stream(lab1 + (size_t)t * S::kLanes + chunk)
                            : make_uint4(0, 0, 0, 0);
+      if (app && t == t_new) {  // the row just appended, from shared memory
+        const uint4* nr = reinterpret_cast<const uint4*>(newrow);
+        v0[i] = nr[(hh * R) / 8 + chunk];
+        if (two) v1[i] = nr[((hh + 1) * R) / 8 + chunk];
+      }
     }
 #pragma unroll
     for (int i = 0; i < S::kSlots; ++i) {

@@ -193,6 +193,24 @@ def test_group_calls_validation():
                                       NUL) == ds.DS_ERR_WORKSPACE
 
 
+def test_group_decode_step_validation():
+    lib = ds.lib()
+    bad = ds.DS_ERR_INVALID_ARG
+    d = _dims(B=2, Hq=8, Hkv=2, T_cap=1000, r=16)
+    args = lambda **kw: [kw.get(n, P) for n in ("Q", "K", "V", "C", "label", "sg", "idx", "O")]
+    assert lib.ds_group_decode_step(*args(sg=NUL), NUL, d, 100, 10, 1.0, 1, NUL, 0, NUL) == bad
+    assert lib.ds_group_decode_step(*args(K=NUL), NUL, d, 100, 10, 1.0, 1, NUL, 0, NUL) == bad
+    assert lib.ds_group_decode_step(*args(), NUL, d, 100, 101, 1.0, 1, NUL, 0, NUL) == bad
+    assert lib.ds_group_decode_step(*args(), NUL, d, 1001, 10, 1.0, 1, NUL, 0, NUL) == bad
+    assert lib.ds_group_decode_step(*args(), NUL, _dims(r=12), 100, 10, 1.0, 1, NUL, 0,
+                                    NUL) == ds.DS_ERR_UNSUPPORTED
+    dl = _dims(B=1, Hq=32, Hkv=8, T_cap=262144, r=8)
+    need = lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384)
+    assert need > 0
+    assert lib.ds_group_decode_step(*args(), NUL, dl, 262144, 16384, 1.0, 1, P, need - 1,
+                                    NUL) == ds.DS_ERR_WORKSPACE
+
+
 def test_block_calls_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG

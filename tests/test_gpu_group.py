@@ -124,3 +124,54 @@ def test_group_full_workload_sampled():
             assert np.abs(On[b, h] - o).max() <= 1e-2
     inp.free()
 
+
+
+STEP_CASES = [
+    # name, B, Hq, Hkv, T, T_cap, r, k, append
+    ("g4-r16", 2, 8, 2, 1000, 1003, 16, 37, True),
+    ("g8-r32", 1, 16, 2, 5000, 5000, 32, 300, True),
+    ("g8-r8-T1", 1, 8, 1, 1, 4, 8, 1, True),
+    ("g2-r128-no-append", 1, 4, 2, 777, 800, 128, 77, False),
+    ("g1-per-head", 2, 4, 4, 3000, 3000, 16, 100, True),
+    ("g16-per-head-kernel", 1, 16, 1, 2000, 2000, 8, 64, True),
+    ("g8-r16-T16384", 2, 16, 2, 16384, 16384, 16, 1024, True),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=[c[0] for c in STEP_CASES])
+def test_group_decode_step_equals_the_three_calls(case):
+    """ds_group_decode_step (the group-score kernel appends token T-1's label rows)
+    gives bit for bit the label cache, group scores, index set, O and lse of
+    ds_label_append + ds_group_score_topk + ds_group_sparse_decode."""
+    name, B, Hq, Hkv, T, T_cap, r, k, append = case
+    w = dsgen.Workload(name, B=B, Hq=Hq, Hkv=Hkv, T=T_cap, r=r, k=k, n_out=min(16, r),
+                       seed=0x6D5 + T)
+    inp = gu.Inputs(w, r=r)
+    label = torch.zeros((B, Hq, T_cap, r), dtype=torch.bfloat16, device="cuda")
+    n0 = T - 1 if append else T
+    if n0 > 0:
+        ds.label_append(inp.dK, inp.dC, label, 0, n0)
+    label_sep = label.clone()
+    if append:
+        ds.label_append(inp.dK, inp.dC, label_sep, T - 1, 1)
+    sg_sep = torch.empty((B * Hkv, T), dtype=torch.float32, device="cuda")
+    idx_sep = torch.empty((B * Hkv, k), dtype=torch.int32, device="cuda")
+    ds.group_score_topk(inp.dQ, inp.dC, label_sep, sg_sep, idx_sep, T)
+    O_sep = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+    L_sep = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ds.group_sparse_decode(inp.dQ, inp.dK, inp.dV, idx_sep, O_sep, T, w.scale, lse=L_sep)
+    sg = torch.full_like(sg_sep, float("nan"))
+    idx = torch.full_like(idx_sep, -1)
+    O = torch.full_like(O_sep, float("nan"))
+    L = torch.full_like(L_sep, float("nan"))
+    ds.group_decode_step(inp.dQ, inp.dK, inp.dV, inp.dC, label, sg, idx, O, T, w.scale,
+                         append=append, lse=L)
+    torch.cuda.synchronize()
+    assert torch.equal(label, label_sep)
+    assert torch.equal(sg, sg_sep)
+    assert torch.equal(idx, idx_sep)
+    assert torch.equal(O, O_sep) and torch.equal(L, L_sep)
+    got_label = gu.host_bits(label)[:, :, :T]
+    assert np.array_equal(got_label, oracle.label(inp.K[:, :, :T], inp.C, Hq))
+    assert ds.device_status() == 0
+    inp.free()
