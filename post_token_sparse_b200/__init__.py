@@ -122,11 +122,11 @@ def _ptr(t: torch.Tensor | None, dtype=None, name="tensor", host_ok=False):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     # K and V (and a decode step's Q, O, lse) may also be pinned host tensors
-    # (see include/ds.h)
+    # (see include/ds.h); whether a host tensor is pinned and mapped is checked by
+    # the library (DS_ERR_INVALID_ARG otherwise), once, on the decode path
     host_ok = host_ok or name in ("K", "V")
-    if not t.is_cuda and not (host_ok and t.is_pinned()):
-        raise TypeError(f"{name} must be a CUDA tensor" +
-                        (" or a pinned host tensor" if host_ok else ""))
+    if not t.is_cuda and not host_ok:
+        raise TypeError(f"{name} must be a CUDA tensor")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
