@@ -944,6 +944,45 @@ def summarize_ncu(src: str) -> None:
          f"gpu_time_ns[k_step]: {dur * 1e3:.0f}"]
     open(os.path.join(prof, f"traffic_{w.name}.txt"), "w").write("\n".join(T) + "\n")
 
+    # the group-by-group attention kernel, when its capture is present
+    grep = os.path.join(src, "k_attend_group_gqa.ncu-rep")
+    if os.path.exists(grep):
+        g = dsgen.workload("gqa-B16-Hq64-Hkv8-T16K")
+        raw = subprocess.run(["ncu", "-i", grep, "--page", "raw", "--csv"], capture_output=True,
+                             text=True, check=True).stdout
+        rr = list(csv.reader(io.StringIO(raw)))
+        h, units, vals = rr[0], rr[1], rr[2]
+        rd, wr = num("dram__bytes_read.sum"), num("dram__bytes_write.sum")
+        dur = num("gpu__time_duration.sum") / (1e3 if get("gpu__time_duration.sum")[1] == "ns"
+                                               else 1)
+        alg = g.dense_bytes()
+        stalls = sorted(((float(vals[i] or 0), m[len(pre):-len(post)]) for i, m in enumerate(h)
+                         if m.startswith(pre) and m.endswith(post) and float(vals[i] or 0) >= 0.05),
+                        reverse=True)
+        gcmd = ("ncu --set full --clock-control none -k regex:k_attend_group -c 1 -o "
+                "k_attend_group_gqa python -m pytest tests/test_gpu_attend_group.py -q -k "
+                "full_gqa_workload_dense")
+        G = [f"# k_attend_group<false> (ds_decode, dense, 8 query heads per KV head), workload "
+             f"{g.name} (B={g.B} Hq={g.Hq} Hkv={g.Hkv} T={g.T})", made, f"#   {gcmd}",
+             "# summarised by: python bench.py --summarize-ncu <dir of the ncu outputs>",
+             "# ncu flushes caches before the captured launch (cold).",
+             f"duration_us (under ncu, cold): {dur:.2f}",
+             f"dram_bytes_read: {rd:.0f}", f"dram_bytes_write: {wr:.0f}",
+             f"algorithmic_bytes_per_launch: {alg}  (K and V once per KV head + Q/O)",
+             f"traffic / algorithmic: {(rd + wr) / alg:.3f}",
+             f"achieved (algorithmic / duration): {alg / dur / 1e3:.0f} GB/s",
+             "dram throughput (% of peak, elapsed): "
+             f"{get('gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed')[0]}",
+             *[f"{m}: {vals[i]}" for i, m in enumerate(h)
+               if "pipe_tensor" in m and "pct_of_peak_sustained" in m][:6],
+             f"registers/thread: {get('launch__registers_per_thread')[0]}  grid: "
+             f"{get('launch__grid_size')[0]}  block: {get('launch__block_size')[0]}",
+             "warps active (% of peak, active cycles): "
+             f"{get('sm__warps_active.avg.pct_of_peak_sustained_active')[0]}",
+             "warp stall reasons (cycles per issued instruction, >= 0.05):"]
+        G += [f"  {n:24s} {v:.2f}" for v, n in stalls]
+        open(os.path.join(prof, f"k_attend_group_{g.name}.txt"), "w").write("\n".join(G) + "\n")
+
 
 def main():
     args = parse()
