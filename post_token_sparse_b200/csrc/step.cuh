@@ -42,6 +42,9 @@ constexpr int kStepTokPerThread = kStepWholeT / kTopkThreads;
 static_assert(kTopkThreads == kSelThreads, "select_whole uses the selector's block scan");
 // shared memory of select_whole, in words: keys, histogram, scan scratch, results
 constexpr int kWholeWords = kStepWholeT + 4096 + 16 + 16;
+// bin tokens ranked by direct counting (above that: the remaining digits by histograms)
+constexpr int kWholeList = 512;
+static_assert(2 * kWholeList + kStepWholeT / 32 <= 4096, "list and bitmap fit the histogram");
 
 struct StepParams {
   const uint16_t* Q;
@@ -296,60 +299,111 @@ __device__ __noinline__ void select_whole(const Grp gr, const uint32_t* keys, ui
   uint32_t* hist = w;             // 4096 bins
   uint32_t* scan = w + 4096;      // 16 words
   uint32_t* res = w + 4096 + 16;  // 16 words
-  uint32_t r = (uint32_t)k, pf = 0u;
-  // digits: (shift, bits) = (20, 12), (8, 12), (0, 8); keys with the prefix pf
-  // above the digit are counted
+  const int t0 = gr.tid() * kStepTokPerThread;  // this thread's tokens t0 .. t0+15
+  // the keys of this thread's tokens, four at a time (f(i, key, valid))
+  auto my_keys = [&](auto&& f) {
 #pragma unroll 1
-  for (int d = 0; d < 3; ++d) {
-    const int sh = d == 0 ? 20 : d == 1 ? 8 : 0;
-    const int nb = d == 2 ? 256 : 4096;
-    const int hs = d == 0 ? 32 : d == 1 ? 20 : 8;  // bits above the digit
-#pragma unroll 1
-    for (int i = gr.tid(); i < nb; i += kTopkThreads) hist[i] = 0u;
-    gr.sync();
-#pragma unroll 1
-    for (int t = gr.tid(); t < T; t += kTopkThreads) {
-      const uint32_t key = keys[t];
-      if (hs >= 32 || (key >> hs) == pf) atomicAdd(&hist[(key >> sh) & (uint32_t)(nb - 1)], 1u);
-    }
-    gr.sync();
-    whole_find_bin(gr, hist, nb, r, scan + 8 * (d & 1), res);
-    pf = (pf << (d == 2 ? 8 : 12)) | res[0];
-    r -= res[1];
-    gr.sync();
-  }
-  const uint32_t thr = pf, need_eq = r;  // the k-th key; ties with it kept: need_eq >= 1
-  // this thread's tokens t0 .. t0+15: keys above thr and equal to it
-  const int t0 = gr.tid() * kStepTokPerThread;
-  uint32_t gt = 0u, eq = 0u;
-#pragma unroll 1
-  for (int i = 0; i < kStepTokPerThread; i += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(keys + t0 + i);
-    const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < kStepTokPerThread; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(keys + t0 + i);
+      const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool ok = t0 + i + u < T;
-      gt |= (uint32_t)(ok && kv[u] > thr) << (i + u);
-      eq |= (uint32_t)(ok && kv[u] == thr) << (i + u);
+      for (int u = 0; u < 4; ++u) f(i + u, kv[u], t0 + i + u < T);
+    }
+  };
+  // first digit (bits 31..20) over every key: the bin b0 of the k-th key
+#pragma unroll 1
+  for (int i = gr.tid(); i < 4096; i += kTopkThreads) hist[i] = 0u;
+  gr.sync();
+#pragma unroll 1
+  for (int t = gr.tid(); t < T; t += kTopkThreads) atomicAdd(&hist[keys[t] >> 20], 1u);
+  gr.sync();
+  whole_find_bin(gr, hist, 4096, (uint32_t)k, scan, res);
+  const uint32_t b0 = res[0];
+  const uint32_t need = (uint32_t)k - res[1];  // keys of bin b0 kept: 1 .. n0
+  const uint32_t n0 = hist[b0];
+  gr.sync();  // every thread has read res and hist[b0]
+  uint32_t keep = 0u;  // this thread's kept tokens
+  if (need == n0) {
+    // every key of bin b0 is kept
+    my_keys([&](int i, uint32_t key, bool ok) { keep |= (uint32_t)(ok && (key >> 20) >= b0) << i; });
+  } else if (n0 <= (uint32_t)kWholeList) {
+    // bin b0's keys listed in token order; each kept when fewer than `need` of
+    // them are larger or equal and earlier (ties to the lower token)
+    uint32_t* lkey = hist;                     // reused: the histogram is read
+    uint32_t* ltok = hist + kWholeList;
+    uint32_t* kept = hist + 2 * kWholeList;    // bitmap of the kept bin tokens
+    uint32_t cm = 0u;
+    my_keys([&](int i, uint32_t key, bool ok) {
+      keep |= (uint32_t)(ok && (key >> 20) > b0) << i;
+      cm |= (uint32_t)(ok && (key >> 20) == b0) << i;
+    });
+    uint32_t tot;
+    uint32_t pos = grp_scan(gr, (uint32_t)__popc(cm), scan + 8, &tot) - (uint32_t)__popc(cm);
+    for (int i = gr.tid(); i < kStepWholeT / 32; i += kTopkThreads) kept[i] = 0u;
+#pragma unroll 1
+    for (uint32_t m = cm; m; m &= m - 1u) {
+      const int i = __ffs(m) - 1;
+      lkey[pos] = keys[t0 + i];
+      ltok[pos] = (uint32_t)(t0 + i);
+      ++pos;
+    }
+    gr.sync();
+#pragma unroll 1
+    for (int i = gr.tid(); i < (int)n0; i += kTopkThreads) {
+      const uint32_t ki = lkey[i];
+      uint32_t ahead = 0u;
+#pragma unroll 4
+      for (int j = 0; j < (int)n0; ++j) {
+        const uint32_t kj = lkey[j];
+        ahead += (uint32_t)(kj > ki || (kj == ki && j < i));
+      }
+      if (ahead < need) atomicOr(&kept[ltok[i] >> 5], 1u << (ltok[i] & 31));
+    }
+    gr.sync();
+    keep |= (kept[t0 >> 5] >> (t0 & 31)) & 0xffffu;
+  } else {
+    // many keys share bin b0: its remaining digits (bits 19..8, then 7..0) by
+    // histograms of the keys that carry the prefix, then the ties in token order
+    uint32_t r = need, pf = b0;
+#pragma unroll 1
+    for (int d = 1; d < 3; ++d) {
+      const int sh = d == 1 ? 8 : 0;
+      const int nb = d == 2 ? 256 : 4096;
+      const int hs = d == 1 ? 20 : 8;  // bits above the digit
+#pragma unroll 1
+      for (int i = gr.tid(); i < nb; i += kTopkThreads) hist[i] = 0u;
+      gr.sync();
+#pragma unroll 1
+      for (int t = gr.tid(); t < T; t += kTopkThreads) {
+        const uint32_t key = keys[t];
+        if ((key >> hs) == pf) atomicAdd(&hist[(key >> sh) & (uint32_t)(nb - 1)], 1u);
+      }
+      gr.sync();
+      whole_find_bin(gr, hist, nb, r, scan + 8 * (d & 1), res);
+      pf = (pf << (d == 2 ? 8 : 12)) | res[0];
+      r -= res[1];
+      gr.sync();
+    }
+    const uint32_t thr = pf, need_eq = r;  // the k-th key; ties with it kept: need_eq >= 1
+    uint32_t eq = 0u;
+    my_keys([&](int i, uint32_t key, bool ok) {
+      keep |= (uint32_t)(ok && key > thr) << i;
+      eq |= (uint32_t)(ok && key == thr) << i;
+    });
+    uint32_t tot;
+    uint32_t rank = grp_scan(gr, (uint32_t)__popc(eq), scan, &tot) - (uint32_t)__popc(eq);
+#pragma unroll 1
+    for (uint32_t m = eq; m; m &= m - 1u) {
+      if (rank < need_eq) keep |= 1u << (__ffs(m) - 1);
+      ++rank;
     }
   }
-  const uint32_t ngt = __popc(gt), neq = __popc(eq);
+  // the kept tokens, ascending
   uint32_t tot;
-  const uint32_t packed = ngt | (neq << 16);
-  const uint32_t excl = grp_scan(gr, packed, scan, &tot) - packed;
-  const uint32_t gt_before = excl & 0xffffu, eq_before = excl >> 16;
-  // the first need_eq ties in token order are kept
-  uint32_t keep = gt, rank = eq_before, m = eq;
-  while (m) {
+  uint32_t pos = grp_scan(gr, (uint32_t)__popc(keep), scan + 8, &tot) - (uint32_t)__popc(keep);
+#pragma unroll 1
+  for (uint32_t m = keep; m; m &= m - 1u) {
     const int i = __ffs(m) - 1;
-    m &= m - 1u;
-    if (rank < need_eq) keep |= 1u << i;
-    ++rank;
-  }
-  uint32_t pos = gt_before + min(eq_before, need_eq);
-  while (keep) {
-    const int i = __ffs(keep) - 1;
-    keep &= keep - 1u;
     dst_s[pos] = t0 + i;
     if (dst_g) dst_g[pos] = t0 + i;
     ++pos;
