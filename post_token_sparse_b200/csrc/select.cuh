@@ -35,7 +35,7 @@ constexpr int kSelThreads = kTopkThreads;  // 8 warps: LabelSource's slicing
 constexpr int kSelTile = 16384;            // tokens scored by one CTA
 constexpr int kSelMaxT = 32768;            // 128 tokens per selector thread at most
 constexpr int kSelMaxRun = kSelMaxT / kSelThreads;
-constexpr int kSelListCap = 2048;          // candidates (and B16's tokens) held in lists
+constexpr int kSelListCap = 4096;          // candidates (and B16's tokens) held in lists
 constexpr int kSelSample = 2048;           // prefixes sampled for the bracket
 constexpr int kSelSlots = 8;               // label loads in flight per thread
 static_assert(kSelThreads == 256, "the selector's scans and 256-bin histograms take 256 threads");
