@@ -234,6 +234,55 @@ struct SelSmem {
   uint32_t selb[kSelMaxT / 32];  // kept tokens found through the lists
 };
 
+// The 16-bit keys of ranks ra and rb (0: not wanted, the output untouched)
+// among the n keys of list[]: both from the same two 8-bit histogram passes.
+__device__ __forceinline__ void blk_select16_pair(const uint16_t* list, int n, uint32_t ra,
+                                                  uint32_t rb, SelSmem& s, uint32_t* out_a,
+                                                  uint32_t* out_b) {
+  uint32_t* h2 = s.ltok;  // [2][256]: the second level of both ranks (free here)
+  s.hist[threadIdx.x] = 0u;
+  h2[threadIdx.x] = 0u;
+  h2[256 + threadIdx.x] = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kSelThreads) atomicAdd(&s.hist[list[i] >> 8], 1u);
+  __syncthreads();
+  // both ranks' bins from one scan
+  const uint32_t c = s.hist[255 - threadIdx.x];
+  uint32_t tot;
+  const uint32_t incl = blk_scan(c, s.scan, &tot);
+  if (c > 0) {
+    if (ra && incl - c < ra && ra <= incl) {
+      s.misc[0] = 255u - threadIdx.x;
+      s.misc[1] = incl - c;
+    }
+    if (rb && incl - c < rb && rb <= incl) {
+      s.misc[4] = 255u - threadIdx.x;
+      s.misc[5] = incl - c;
+    }
+  }
+  __syncthreads();
+  const uint32_t ba = s.misc[0], aa = s.misc[1], bb = s.misc[4], ab = s.misc[5];
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t key = list[i];
+    if (ra && (key >> 8) == ba) atomicAdd(&h2[key & 255u], 1u);
+    if (rb && (key >> 8) == bb) atomicAdd(&h2[256 + (key & 255u)], 1u);
+  }
+  __syncthreads();
+  const uint32_t ca = h2[255 - threadIdx.x], cb = h2[256 + 255 - threadIdx.x];
+  const uint32_t inca = blk_scan(ca, s.scan + 8, &tot);
+  __syncthreads();
+  const uint32_t incb = blk_scan(cb, s.scan, &tot);
+  if (ra && ca > 0 && inca - ca < ra - aa && ra - aa <= inca) *out_a = (ba << 8) | (255u - threadIdx.x);
+  if (rb && cb > 0 && incb - cb < rb - ab && rb - ab <= incb) *out_b = (bb << 8) | (255u - threadIdx.x);
+  // every thread takes the results from the two that found them
+  if (ra && ca > 0 && inca - ca < ra - aa && ra - aa <= inca) s.misc[2] = *out_a;
+  if (rb && cb > 0 && incb - cb < rb - ab && rb - ab <= incb) s.misc[6] = *out_b;
+  __syncthreads();
+  if (ra) *out_a = s.misc[2];
+  if (rb) *out_b = s.misc[6];
+  __syncthreads();
+}
+
 // Selection of head bh from its prefixes, by the whole CTA; ks gives the exact
 // keys of the boundary bin's tokens.
 template <class KS>
@@ -266,10 +315,9 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
     for (int j = 0; j < kSelSample / kSelThreads; ++j) s.smp[threadIdx.x + j * kSelThreads] = v[j];
   }
   __syncthreads();
-  auto sample = [&](int i) { return (uint32_t)s.smp[i]; };
-  uint32_t hi = 0xffffffffu, lo = 0u, ua, ue;
-  if (r_hi >= 1) hi = blk_select16(sample, mv, (uint32_t)r_hi, s.hist, s.scan, s.misc, &ua, &ue);
-  if (r_lo <= mv) lo = blk_select16(sample, mv, (uint32_t)r_lo, s.hist, s.scan, s.misc, &ua, &ue);
+  uint32_t hi = 0xffffffffu, lo = 0u;
+  blk_select16_pair(s.smp, mv, r_hi >= 1 ? (uint32_t)r_hi : 0u, r_lo <= mv ? (uint32_t)r_lo : 0u,
+                    s, &hi, &lo);
 
   // 2. register masks of this thread's run: above the bracket, inside it
   uint32_t am[4] = {0u, 0u, 0u, 0u}, cm[4] = {0u, 0u, 0u, 0u};
