@@ -667,7 +667,7 @@ def group_entry(w, inputs, hbm_peak, steps: int = 50):
     sg = torch.empty((w.B * w.Hkv, w.T), dtype=torch.float32, device="cuda")
     idx = torch.empty((w.B * w.Hkv, w.k), dtype=torch.int32, device="cuda")
     O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
-    ws = ds.workspace(ds.OP_GROUP_SPARSE_DECODE, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
+    ws = ds.workspace(ds.OP_GROUP_DECODE_STEP, ds.dims_of(Q, K, w.r), w.T, w.k, "cuda")
 
     def step():
         ds.group_decode_step(Q, K, V, C, label, sg, idx, O, w.T, w.scale, ws=ws)

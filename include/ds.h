@@ -92,7 +92,8 @@ enum {
   DS_OP_DECODE_STEP = 6,
   DS_OP_CALIBRATE = 7, /* k: calibration queries per head (Nq) */
   DS_OP_GROUP_SPARSE_DECODE = 8,
-  DS_OP_BLOCK_SPARSE_DECODE = 9 /* k: kept rows = kb * bs */
+  DS_OP_BLOCK_SPARSE_DECODE = 9, /* k: kept rows = kb * bs */
+  DS_OP_GROUP_DECODE_STEP = 10
 };
 
 /* Device status bits (ds_device_status). */
@@ -158,8 +159,14 @@ ds_status ds_score(const void* Q, const int32_t* C, const void* label, float* sc
  * the contract (no fault, unspecified choice).  Token selection by the higher
  * activation (Double Sparsity page, Method details: Key design).
  *
- * Requires 1 <= k <= T <= 1048576 and BH <= 65535.  Needs no workspace
- * (ds_workspace_size returns 0); `ws` may be NULL.
+ * Requires 1 <= k <= T <= 1048576 and BH <= 65535.  ws: NULL, or
+ * ds_workspace_size(DS_OP_TOPK, dims, T, k) bytes (dims.B * dims.Hq = BH) of
+ * 16-byte aligned device memory, zero-filled before first use (its counters
+ * are left at zero).  When that size is nonzero (4096 < T <= 16384) and ws
+ * is given, one launch turns tiles of 4096 scores into 16-bit key prefixes
+ * and the last tile of each row selects from them (exact keys from the
+ * scores); otherwise the selection kernel reads the scores directly.  Same
+ * result either way.
  */
 ds_status ds_topk(const float* scores, int32_t* idx, int32_t BH, int32_t T, int32_t k,
                   void* ws, size_t ws_bytes, ds_stream_t stream);
@@ -362,9 +369,10 @@ ds_status ds_group_sparse_decode(const void* Q, const void* K, const void* V,
  * from them.  Results identical to the three calls.
  *
  * Arguments as for those calls (label written at T-1 when append != 0).  ws:
- * ds_workspace_size(DS_OP_GROUP_SPARSE_DECODE, dims, T, k) bytes, zero-filled
- * before first use.  Requires what ds_group_score_topk requires, with
- * G*r*6 <= 49152.
+ * ds_workspace_size(DS_OP_GROUP_DECODE_STEP, dims, T, k) bytes, zero-filled
+ * before first use: the attention's workspace, then, for 4096 < T <= 16384,
+ * that of the one-launch top-k over the group scores (as ds_topk's).
+ * Requires what ds_group_score_topk requires, with G*r*6 <= 49152.
  */
 ds_status ds_group_decode_step(const void* Q, const void* K, const void* V, const int32_t* C,
                                void* label, float* group_scores, int32_t* idx, float* O,

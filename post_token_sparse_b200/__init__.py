@@ -33,7 +33,8 @@ LIB_PATH = os.path.join(_HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_WORKSPACE, DS_ERR_CUDA = range(5)
 (OP_LABEL_APPEND, OP_SCORE, OP_TOPK, OP_SPARSE_DECODE, OP_DECODE, OP_SCORE_TOPK,
- OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE) = range(10)
+ OP_DECODE_STEP, OP_CALIBRATE, OP_GROUP_SPARSE_DECODE, OP_BLOCK_SPARSE_DECODE,
+ OP_GROUP_DECODE_STEP) = range(11)
 DEV_BAD_CHANNEL, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
 
 
@@ -196,13 +197,19 @@ def score(Q, C, label, scores, T: int):
                          dims, T, _stream(Q.device)), "ds_score")
 
 
-def topk(scores, idx):
+def topk(scores, idx, ws=None):
+    """Top-k of each row of scores [BH, T] into idx [BH, k]; ws: the workspace of
+    OP_TOPK (made here when not given)."""
     BH, T = scores.shape
     k = idx.shape[-1]
     if idx.numel() != BH * k:
         raise TypeError("idx must have BH*k elements")
+    if ws is None:
+        ws = workspace(OP_TOPK, Dims(1, BH, 1, 128, T, 1), T, k, scores.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(_lib.ds_topk(_ptr(scores, torch.float32, "scores"), _ptr(idx, torch.int32, "idx"),
-                        BH, T, k, None, 0, _stream(scores.device)), "ds_topk")
+                        BH, T, k, _ptr(ws, None, "ws"), nbytes, _stream(scores.device)),
+           "ds_topk")
 
 
 def score_topk(Q, C, label, idx, T: int, scores=None, ws=None):
@@ -306,7 +313,7 @@ def group_decode_step(Q, K, V, C, label, group_scores, idx, O, T: int, scale: fl
     dims = Dims(B, Hq, Hkv, Q.shape[-1], T_cap, r)
     k = idx.shape[-1]
     if ws is None:
-        ws = workspace(OP_GROUP_SPARSE_DECODE, dims, T, k, Q.device)
+        ws = workspace(OP_GROUP_DECODE_STEP, dims, T, k, Q.device)
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(_lib.ds_group_decode_step(
         _ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),

@@ -128,8 +128,9 @@ __device__ __forceinline__ void exact_keys(const uint16_t* lab, const float* qs,
   }
 }
 
-// Exact keys of a head's tokens for the selection's boundary bin, recomputed
-// from the head's label rows.
+// Exact keys of a head's tokens for the selection's boundary bin: recomputed
+// from the head's label rows (LabelKeys), or read from written scores
+// (StoredKeys).
 template <int R>
 struct LabelKeys {
   const uint16_t* lab;
@@ -141,6 +142,27 @@ struct LabelKeys {
     exact_keys<R>(lab, qs, tok, key, n);
   }
 };
+struct StoredKeys {
+  const float* sc;  // the head's scores; read around L1 (another kernel may have written them)
+  __device__ __forceinline__ uint32_t key(int t) const { return order_key(__ldcg(sc + t)); }
+  __device__ __forceinline__ void keys(const uint32_t* tok, uint32_t* key, int n) const {
+    constexpr int kB = 4;
+    for (int i0 = threadIdx.x; i0 < n; i0 += kB * kSelThreads) {
+      float v[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int i = i0 + j * kSelThreads;
+        v[j] = i < n ? __ldcg(sc + tok[i]) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int i = i0 + j * kSelThreads;
+        if (i < n) key[i] = order_key(v[j]);
+      }
+    }
+  }
+};
+
 // Inclusive prefix over the CTA's threads in order; *total: the sum.
 // scratch: 8 words, not rewritten before the caller's next barrier.
 __device__ __forceinline__ uint32_t blk_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
@@ -567,6 +589,38 @@ k_score_select(const SelParams p) {
   if (s.misc[S_LAST] == 0u) return;
   __threadfence();
   select_head(p, bh, s, LabelKeys<R>{p.label + (size_t)bh * p.T_cap * R, s.qs});
+  if (threadIdx.x == 0) p.arrivals[bh] = 0u;  // zero again for the next call
+}
+
+// ---- top-k over written scores in one launch ---------------------------------
+//
+// The same selection over a [BH, T] score array (ds_topk's contract): grid
+// (ceil(T / kScoresTile), BH); each CTA turns one tile of scores into 16-bit
+// key prefixes, and the head's last tile selects, taking the boundary bin's
+// exact keys from the scores.  The scores are small (4 bytes a token), so the
+// tiles are short and the selections of all heads overlap.
+constexpr int kScoresTile = 4096;
+
+__global__ void __launch_bounds__(kSelThreads, 3)
+k_scores_select(const SelParams p) {
+  __shared__ SelSmem s;
+  const int bh = blockIdx.y;
+  const int T = p.T, per = sel_per(T);
+  uint16_t* pref = p.prefixes + (size_t)bh * per * kSelThreads;
+  const float* sc = p.scores + (size_t)bh * T;
+  const int t_end = min(T, (int)(blockIdx.x + 1) * kScoresTile);
+#pragma unroll 4
+  for (int t = blockIdx.x * kScoresTile + threadIdx.x; t < t_end; t += kSelThreads)
+    pref[key_slot(t, per)] = (uint16_t)(order_key(__ldg(sc + t)) >> 16);
+  // the head's last tile to finish selects it
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    s.misc[S_LAST] = atomicAdd(&p.arrivals[bh], 1u) == gridDim.x - 1 ? 1u : 0u;
+  __syncthreads();
+  if (s.misc[S_LAST] == 0u) return;
+  __threadfence();
+  select_head(p, bh, s, StoredKeys{sc});
   if (threadIdx.x == 0) p.arrivals[bh] = 0u;  // zero again for the next call
 }
 

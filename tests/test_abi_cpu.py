@@ -131,9 +131,11 @@ def test_workspace_sizes():
     # short rows: every warp takes whole heads, nothing to merge, no workspace
     d = _dims(B=32, Hq=32, Hkv=32, T_cap=32768, r=8)
     assert lib.ds_workspace_size(ds.OP_SPARSE_DECODE, d, 32768, 16) == 0
-    assert lib.ds_workspace_size(ds.OP_TOPK, d, 32768, 512) == 0
-    # the one-launch selection keeps 2-byte key prefixes of every token (T_pad a
+    # the one-launch selections keep 2-byte key prefixes of every token (T_pad a
     # power of two times 256) after 256 KiB of counters
+    assert lib.ds_workspace_size(ds.OP_TOPK, d, 16384, 512) == 256 * 1024 + 32 * 32 * 16384 * 2
+    assert lib.ds_workspace_size(ds.OP_TOPK, d, 4096, 512) == 0
+    assert lib.ds_workspace_size(ds.OP_TOPK, d, 16385, 512) == 0
     assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 32768, 512) == \
         256 * 1024 + 32 * 32 * 32768 * 2
     assert lib.ds_workspace_size(ds.OP_SCORE_TOPK, d, 4096, 512) == 0  # one CTA per head
@@ -193,6 +195,18 @@ def test_group_calls_validation():
                                       NUL) == ds.DS_ERR_WORKSPACE
 
 
+def test_group_decode_step_workspace():
+    """The attention's workspace, then (4096 < T <= 16384) the one-launch top-k's
+    over the group scores, 256-byte aligned."""
+    lib = ds.lib()
+    d = _dims(B=16, Hq=64, Hkv=8, T_cap=16384, r=16)
+    att = lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, d, 16384, 1024)
+    want = (att + 255) // 256 * 256 + 256 * 1024 + 128 * 16384 * 2
+    assert lib.ds_workspace_size(ds.OP_GROUP_DECODE_STEP, d, 16384, 1024) == want
+    assert lib.ds_workspace_size(ds.OP_GROUP_DECODE_STEP, d, 4096, 256) == \
+        lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, d, 4096, 256)
+
+
 def test_group_decode_step_validation():
     lib = ds.lib()
     bad = ds.DS_ERR_INVALID_ARG
@@ -205,7 +219,7 @@ def test_group_decode_step_validation():
     assert lib.ds_group_decode_step(*args(), NUL, _dims(r=12), 100, 10, 1.0, 1, NUL, 0,
                                     NUL) == ds.DS_ERR_UNSUPPORTED
     dl = _dims(B=1, Hq=32, Hkv=8, T_cap=262144, r=8)
-    need = lib.ds_workspace_size(ds.OP_GROUP_SPARSE_DECODE, dl, 262144, 16384)
+    need = lib.ds_workspace_size(ds.OP_GROUP_DECODE_STEP, dl, 262144, 16384)
     assert need > 0
     assert lib.ds_group_decode_step(*args(), NUL, dl, 262144, 16384, 1.0, 1, P, need - 1,
                                     NUL) == ds.DS_ERR_WORKSPACE

@@ -93,3 +93,36 @@ def test_score_select_few_distinct_scores(T, k, kmod):
 def test_score_select_all_scores_equal():
     """Q = 0: every score is +0 (or -0, equal to it): the first k tokens."""
     _run(16, 32, 32, 10000, 8, 4321, seed=99, zero_q=True)
+
+
+@pytest.mark.parametrize("BH,T,k,mode", [(6, 4097, 1, "normal"), (5, 16384, 1024, "ints"),
+                                         (3, 16384, 8192, "normal"), (4, 12000, 11999, "ints"),
+                                         (2, 9000, 700, "zero")])
+def test_topk_over_scores_one_launch_equals_plain(BH, T, k, mode):
+    """ds_topk with a workspace (tiles of written scores into key prefixes, the
+    row's last tile selects) gives the index set of the call without one, and
+    the oracle's rule on the same scores (ties to the lower index)."""
+    import ctypes
+    rng = np.random.default_rng(T + k)
+    if mode == "ints":
+        S = rng.integers(-20, 21, size=(BH, T)).astype(np.float32)
+    elif mode == "zero":
+        S = np.zeros((BH, T), np.float32)
+        S[:, ::7] = -0.0
+    else:
+        S = (rng.standard_normal((BH, T)) * 40).astype(np.float32)
+    sc = torch.from_numpy(S).cuda()
+    i_ws = torch.full((BH, k), -1, dtype=torch.int32, device="cuda")
+    ds.topk(sc, i_ws)  # the binding makes the workspace
+    ws_bytes = ds.workspace_size(ds.OP_TOPK, ds.Dims(1, BH, 1, 128, T, 1), T, k)
+    assert ws_bytes > 0
+    i_plain = torch.full_like(i_ws, -1)
+    st = ds.lib().ds_topk(ctypes.c_void_p(sc.data_ptr()), ctypes.c_void_p(i_plain.data_ptr()),
+                          BH, T, k, None, 0,
+                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == ds.DS_OK
+    torch.cuda.synchronize()
+    assert torch.equal(i_ws, i_plain)
+    I = i_ws.cpu().numpy()
+    for b in range(BH):
+        assert np.array_equal(I[b], oracle.topk_head(S[b], k)), b
