@@ -103,3 +103,37 @@ def test_decode_step_with_query_and_output_in_host_memory(shape):
         assert torch.equal(a.cpu(), b.cpu())
     assert ds.device_status() == 0
     inp.free()
+
+
+@pytest.mark.parametrize("shape", [(2, 16, 2, 9000, 16, 600), (1, 8, 2, 3000, 8, 100)],
+                         ids=["g8-T9000", "g4-T3000"])
+def test_group_decode_step_with_offloaded_kv(shape):
+    """ds_group_decode_step with K and V in page-locked host memory (the label
+    append reads the new token's channels and the attention the kept rows over
+    the host link) gives the bits of the device-resident run."""
+    B, Hq, Hkv, T, r, k = shape
+    w = dsgen.Workload("offload-group", B=B, Hq=Hq, Hkv=Hkv, T=T, r=r, k=k, n_out=min(16, r),
+                       seed=0x6F1 + T)
+    inp = gu.Inputs(w)
+    hK, hV = _pinned(inp.K), _pinned(inp.V)
+
+    def run(K, V):
+        label = torch.zeros((B, Hq, T, r), dtype=torch.bfloat16, device="cuda")
+        ds.label_append(inp.dK, inp.dC, label, 0, T - 1)
+        sg = torch.empty((B * Hkv, T), dtype=torch.float32, device="cuda")
+        idx = torch.empty((B * Hkv, k), dtype=torch.int32, device="cuda")
+        O = torch.empty((B, Hq, w.d), dtype=torch.float32, device="cuda")
+        L = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        ds.group_decode_step(inp.dQ, K, V, inp.dC, label, sg, idx, O, T, w.scale, lse=L)
+        torch.cuda.synchronize()
+        return label, sg, idx, O, L
+
+    dev = run(inp.dK, inp.dV)
+    host = run(hK, hV)
+    for a, b in zip(dev, host):
+        assert torch.equal(a, b)
+    I = host[2].cpu().numpy().reshape(B, Hkv, k)
+    ref_O, _ = oracle.group_attend(inp.Q, inp.K, inp.V, I, w.scale)
+    assert np.abs(host[3].cpu().numpy() - ref_O).max() <= 1e-2
+    assert ds.device_status() == 0
+    inp.free()
