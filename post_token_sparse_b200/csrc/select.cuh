@@ -245,14 +245,19 @@ __device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f)
   }
 }
 
+// Per-thread candidate entries kept during the mask pass: (16-bit key << 16) |
+// offset in the run, entry c of thread t at word c * kSelThreads + t, in the
+// candidate lists' storage (free until the boundary bin is known).
+constexpr int kSelOwnCands = 2 * kSelListCap / kSelThreads;  // 32
+
 struct SelSmem {
   float qs[128];
   uint32_t hist[256];
   uint32_t misc[8];
   uint32_t scan[16];
   uint16_t smp[kSelSample];  // the bracket's subsample of prefixes
-  uint32_t ltok[kSelListCap];
-  uint32_t lkey[kSelListCap];
+  uint32_t ltok[kSelListCap];  // ltok and lkey adjacent: the candidate entries
+  uint32_t lkey[kSelListCap];  // of the mask pass use both
   uint32_t selb[kSelMaxT / 32];  // kept tokens found through the lists
 };
 
@@ -341,12 +346,20 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
   blk_select16_pair(s.smp, mv, r_hi >= 1 ? (uint32_t)r_hi : 0u, r_lo <= mv ? (uint32_t)r_lo : 0u,
                     s, &hi, &lo);
 
-  // 2. register masks of this thread's run: above the bracket, inside it
+  // 2. register masks of this thread's run: above the bracket, inside it; the
+  // candidates (inside it) also kept as entries of this thread
   uint32_t am[4] = {0u, 0u, 0u, 0u}, cm[4] = {0u, 0u, 0u, 0u};
+  uint32_t* own = s.ltok;  // kSelOwnCands entries a thread (ltok, then lkey)
+  uint32_t n_own = 0;
   for_my_run(pref, per, [&](int j, uint32_t key) {
     const bool v = in_t(j);
+    const bool c = v && key >= lo && key <= hi;
     am[j >> 5] |= (uint32_t)(v && key > hi) << (j & 31);
-    cm[j >> 5] |= (uint32_t)(v && key >= lo && key <= hi) << (j & 31);
+    cm[j >> 5] |= (uint32_t)c << (j & 31);
+    if (c) {
+      if (n_own < (uint32_t)kSelOwnCands) own[n_own * kSelThreads + threadIdx.x] = (key << 16) | j;
+      ++n_own;
+    }
   });
   const uint32_t na = __popc(am[0]) + __popc(am[1]) + __popc(am[2]) + __popc(am[3]);
   const uint32_t nc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
@@ -354,11 +367,50 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
   const uint32_t incl = blk_scan(na | (nc << 16), s.scan, &tot);
   const uint32_t n_above = tot & 0xffffu, n_cand = tot >> 16;
   const bool listed = n_cand <= (uint32_t)kSelListCap && n_above < k && k <= n_above + n_cand;
+  // every thread kept all its candidates as entries: the bin B16 is found from
+  // them, without reading the prefixes again
+  const bool owned = listed && !__syncthreads_or(nc > (uint32_t)kSelOwnCands);
   __syncthreads();
 
   // 3. the bin B16 of the k-th key
   uint32_t B16, ngt16, neq;
-  if (listed) {
+  uint32_t bm[4] = {0u, 0u, 0u, 0u};  // this thread's tokens of B16
+  auto set_bit = [](uint32_t (&m)[4], int j) {
+    const uint32_t b = 1u << (j & 31);
+    const int w = j >> 5;
+    m[0] |= w == 0 ? b : 0u;
+    m[1] |= w == 1 ? b : 0u;
+    m[2] |= w == 2 ? b : 0u;
+    m[3] |= w == 3 ? b : 0u;
+  };
+  if (owned) {
+    // two 8-bit levels over the entries, each thread adding its own
+    s.hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for (uint32_t c = 0; c < nc; ++c) atomicAdd(&s.hist[own[c * kSelThreads + threadIdx.x] >> 24], 1u);
+    __syncthreads();
+    blk_find_bin(s.hist, k - n_above, s.scan, s.misc);
+    const uint32_t b1 = s.misc[S_BIN], a1 = s.misc[S_ABV];
+    s.hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for (uint32_t c = 0; c < nc; ++c) {
+      const uint32_t e = own[c * kSelThreads + threadIdx.x];
+      if ((e >> 24) == b1) atomicAdd(&s.hist[(e >> 16) & 255u], 1u);
+    }
+    __syncthreads();
+    blk_find_bin(s.hist, k - n_above - a1, s.scan + 8, s.misc);
+    B16 = (b1 << 8) | s.misc[S_BIN];
+    ngt16 = n_above + a1 + s.misc[S_ABV];
+    neq = s.misc[S_CNT];
+    // this thread's candidates above B16 join its mask; those in B16 are marked
+    for (uint32_t c = 0; c < nc; ++c) {
+      const uint32_t e = own[c * kSelThreads + threadIdx.x];
+      const uint32_t key16 = e >> 16;
+      const int j = (int)(e & 0xffffu);
+      if (key16 > B16) set_bit(am, j);
+      if (key16 == B16) set_bit(bm, j);
+    }
+  } else if (listed) {
     // the candidates in token order: the 16-byte prefix words that hold any are
     // loaded again, all at once
     uint32_t pos = (incl - (na | (nc << 16))) >> 16;
@@ -419,8 +471,9 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
 
   // 4. B16's tokens: all kept, or the exact threshold among them
   const uint32_t need = k - ngt16;  // 1 <= need <= neq
-  uint32_t bm[4] = {0u, 0u, 0u, 0u};  // this thread's tokens of B16
-  if (listed) {
+  if (owned) {
+    // marked above
+  } else if (listed) {
     // B16 lies inside the bracket: its tokens are candidates of this thread's
     // own run, in the list slice this thread wrote
     const uint32_t pos0 = (incl - (na | (nc << 16))) >> 16;
