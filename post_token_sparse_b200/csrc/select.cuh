@@ -230,17 +230,32 @@ __device__ __forceinline__ uint32_t blk_select16(KeyOf key_of, int n, uint32_t r
 
 // Calls f(j, prefix) for j = 0 .. per-1 of this thread's run (j: the token's
 // offset in the run), eight prefixes per 16-byte load, read around L1 (the
-// prefixes were written by other CTAs).
+// prefixes were written by other CTAs).  The loads go out in batches of four
+// before any prefix is used: while the SM's other CTAs stream, an L2 round trip
+// takes about a microsecond, and f's shared-memory stores would otherwise keep
+// each load behind the previous word's work.
+constexpr int kRunBatch = 4;
+
 template <class F>
 __device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f) {
   const uint4* p4 = reinterpret_cast<const uint4*>(pref);
+  const int words = per / 8;
 #pragma unroll
-  for (int i = 0; i < kSelMaxRun / 8; ++i) {
-    if (i < per / 8) {
-      const uint4 v = __ldcg(p4 + i * kSelThreads + threadIdx.x);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  for (int i0 = 0; i0 < kSelMaxRun / 8; i0 += kRunBatch) {
+    if (i0 < words) {
+      uint4 v[kRunBatch];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f(8 * i + e, (w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+      for (int b = 0; b < kRunBatch; ++b)
+        v[b] = i0 + b < words ? __ldcg(p4 + (i0 + b) * kSelThreads + threadIdx.x)
+                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int b = 0; b < kRunBatch; ++b) {
+        if (i0 + b < words) {
+          const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f(8 * (i0 + b) + e, (w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+        }
+      }
     }
   }
 }
