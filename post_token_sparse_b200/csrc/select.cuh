@@ -36,6 +36,7 @@ constexpr int kSelTile = 16384;            // tokens scored by one CTA
 constexpr int kSelMaxT = 32768;            // 128 tokens per selector thread at most
 constexpr int kSelMaxRun = kSelMaxT / kSelThreads;
 constexpr int kSelListCap = 4096;          // candidates (and B16's tokens) held in lists
+constexpr int kSelSmallBin = 64;           // B16's tokens ranked by one warp up to this
 constexpr int kSelSample = 2048;           // prefixes sampled for the bracket
 constexpr int kSelSlots = 8;               // label loads in flight per thread
 static_assert(kSelThreads == 256, "the selector's scans and 256-bin histograms take 256 threads");
@@ -521,21 +522,40 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
     __syncthreads();
     ks.keys(s.ltok, s.lkey, (int)neq);
     __syncthreads();
-    uint32_t above_e, eq_e;
-    const uint32_t thr =
-        (B16 << 16) | blk_select16([&](int i) { return s.lkey[i]; }, (int)neq, need, s.hist,
-                                   s.scan, s.misc, &above_e, &eq_e);
-    const uint32_t need_eq = need - above_e;
-    const int per_t = ((int)neq + kSelThreads - 1) / kSelThreads;
-    const int s0 = min((int)threadIdx.x * per_t, (int)neq), s1 = min(s0 + per_t, (int)neq);
-    uint32_t nt = 0;
-    for (int i = s0; i < s1; ++i) nt += s.lkey[i] == thr;
-    uint32_t rank = blk_scan(nt, s.scan, &tot) - nt;
-    for (int i = s0; i < s1; ++i) {
-      const uint32_t key = s.lkey[i], t = s.ltok[i];
-      bool keep = key > thr;
-      if (key == thr) keep = rank++ < need_eq;
-      if (keep) atomicOr(&s.selb[t >> 5], 1u << (t & 31));
+    if (neq <= (uint32_t)kSelSmallBin) {
+      // few tokens: one warp ranks each by the keys above it and the equal keys
+      // before it in token order, and keeps the need first
+      if (threadIdx.x < 32) {
+        for (uint32_t i = threadIdx.x; i < neq; i += 32) {
+          const uint32_t ki = s.lkey[i];
+          uint32_t rank = 0;
+          for (uint32_t j = 0; j < neq; ++j) {
+            const uint32_t kj = s.lkey[j];
+            rank += (uint32_t)(kj > ki) | ((uint32_t)(kj == ki) & (uint32_t)(j < i));
+          }
+          if (rank < need) {
+            const uint32_t t = s.ltok[i];
+            atomicOr(&s.selb[t >> 5], 1u << (t & 31));
+          }
+        }
+      }
+    } else {
+      uint32_t above_e, eq_e;
+      const uint32_t thr =
+          (B16 << 16) | blk_select16([&](int i) { return s.lkey[i]; }, (int)neq, need, s.hist,
+                                     s.scan, s.misc, &above_e, &eq_e);
+      const uint32_t need_eq = need - above_e;
+      const int per_t = ((int)neq + kSelThreads - 1) / kSelThreads;
+      const int s0 = min((int)threadIdx.x * per_t, (int)neq), s1 = min(s0 + per_t, (int)neq);
+      uint32_t nt = 0;
+      for (int i = s0; i < s1; ++i) nt += s.lkey[i] == thr;
+      uint32_t rank = blk_scan(nt, s.scan, &tot) - nt;
+      for (int i = s0; i < s1; ++i) {
+        const uint32_t key = s.lkey[i], t = s.ltok[i];
+        bool keep = key > thr;
+        if (key == thr) keep = rank++ < need_eq;
+        if (keep) atomicOr(&s.selb[t >> 5], 1u << (t & 31));
+      }
     }
   } else {
     // more tokens in B16 than the list holds: exact keys recomputed in place
