@@ -237,8 +237,10 @@ __device__ __forceinline__ uint32_t blk_select16(KeyOf key_of, int n, uint32_t r
 // each load behind the previous word's work.
 constexpr int kRunBatch = 4;
 
+// Calls f(i, w) for each 16-byte word i = 0 .. per/8-1 of this thread's run: w
+// holds the prefixes of tokens 8i .. 8i+7, two a word, the lower token low.
 template <class F>
-__device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f) {
+__device__ __forceinline__ void for_my_words(const uint16_t* pref, int per, F&& f) {
   const uint4* p4 = reinterpret_cast<const uint4*>(pref);
   const int words = per / 8;
 #pragma unroll
@@ -253,12 +255,19 @@ __device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f)
       for (int b = 0; b < kRunBatch; ++b) {
         if (i0 + b < words) {
           const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f(8 * (i0 + b) + e, (w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+          f(i0 + b, w);
         }
       }
     }
   }
+}
+
+template <class F>
+__device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f) {
+  for_my_words(pref, per, [&](int i, const uint32_t (&w)[4]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f(8 * i + e, (w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+  });
 }
 
 // Per-thread candidate entries kept during the mask pass: (16-bit key << 16) |
@@ -367,16 +376,40 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
   uint32_t am[4] = {0u, 0u, 0u, 0u}, cm[4] = {0u, 0u, 0u, 0u};
   uint32_t* own = s.ltok;  // kSelOwnCands entries a thread (ltok, then lkey)
   uint32_t n_own = 0;
-  for_my_run(pref, per, [&](int j, uint32_t key) {
-    const bool v = in_t(j);
-    const bool c = v && key >= lo && key <= hi;
-    am[j >> 5] |= (uint32_t)(v && key > hi) << (j & 31);
-    cm[j >> 5] |= (uint32_t)c << (j & 31);
-    if (c) {
-      if (n_own < (uint32_t)kSelOwnCands) own[n_own * kSelThreads + threadIdx.x] = (key << 16) | j;
+  const uint32_t span = hi - lo;  // lo <= hi: the candidates are key - lo <= span
+  for_my_words(pref, per, [&](int i, const uint32_t (&w)[4]) {
+    uint32_t g8 = 0u, c8 = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t key = (w[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+      g8 |= (uint32_t)(key > hi) << e;
+      c8 |= (uint32_t)(key - lo <= span) << e;
+    }
+    am[i >> 2] |= g8 << (8 * (i & 3));
+    cm[i >> 2] |= c8 << (8 * (i & 3));
+    while (c8) {  // the word's candidates (a few percent of the tokens) as entries
+      const int e = __ffs(c8) - 1;
+      c8 &= c8 - 1u;
+      const int q = e >> 1;
+      const uint32_t ww = q == 0 ? w[0] : q == 1 ? w[1] : q == 2 ? w[2] : w[3];
+      const uint32_t key = (ww >> (16 * (e & 1))) & 0xffffu;
+      if (n_own < (uint32_t)kSelOwnCands)
+        own[n_own * kSelThreads + threadIdx.x] = (key << 16) | (uint32_t)(8 * i + e);
       ++n_own;
     }
   });
+  // tokens at or past T (stale prefix slots) leave both masks; entries made for
+  // them follow the valid ones and are never read (nc counts valid ones only)
+  {
+    const int nv = T - t0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int nb = nv - 32 * w;
+      const uint32_t vm = nb >= 32 ? 0xffffffffu : nb <= 0 ? 0u : (1u << nb) - 1u;
+      am[w] &= vm;
+      cm[w] &= vm;
+    }
+  }
   const uint32_t na = __popc(am[0]) + __popc(am[1]) + __popc(am[2]) + __popc(am[3]);
   const uint32_t nc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
   uint32_t tot;
@@ -399,7 +432,18 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
     m[2] |= w == 2 ? b : 0u;
     m[3] |= w == 3 ? b : 0u;
   };
-  if (owned) {
+  if (owned && hi - lo < 256u) {
+    // the bracket spans fewer than 256 prefix values: one histogram of key - lo
+    s.hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for (uint32_t c = 0; c < nc; ++c)
+      atomicAdd(&s.hist[(own[c * kSelThreads + threadIdx.x] >> 16) - lo], 1u);
+    __syncthreads();
+    blk_find_bin(s.hist, k - n_above, s.scan, s.misc);
+    B16 = lo + s.misc[S_BIN];
+    ngt16 = n_above + s.misc[S_ABV];
+    neq = s.misc[S_CNT];
+  } else if (owned) {
     // two 8-bit levels over the entries, each thread adding its own
     s.hist[threadIdx.x] = 0u;
     __syncthreads();
@@ -418,6 +462,8 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
     B16 = (b1 << 8) | s.misc[S_BIN];
     ngt16 = n_above + a1 + s.misc[S_ABV];
     neq = s.misc[S_CNT];
+  }
+  if (owned) {
     // this thread's candidates above B16 join its mask; those in B16 are marked
     for (uint32_t c = 0; c < nc; ++c) {
       const uint32_t e = own[c * kSelThreads + threadIdx.x];

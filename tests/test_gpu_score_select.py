@@ -97,7 +97,8 @@ def test_score_select_all_scores_equal():
 
 @pytest.mark.parametrize("BH,T,k,mode", [(6, 4097, 1, "normal"), (5, 16384, 1024, "ints"),
                                          (3, 16384, 8192, "normal"), (4, 12000, 11999, "ints"),
-                                         (2, 9000, 700, "zero")])
+                                         (2, 9000, 700, "zero"), (4, 16384, 1024, "wide"),
+                                         (3, 16000, 300, "wide")])
 def test_topk_over_scores_one_launch_equals_plain(BH, T, k, mode):
     """ds_topk with a workspace (tiles of written scores into key prefixes, the
     row's last tile selects) gives the index set of the call without one, and
@@ -109,6 +110,11 @@ def test_topk_over_scores_one_launch_equals_plain(BH, T, k, mode):
     elif mode == "zero":
         S = np.zeros((BH, T), np.float32)
         S[:, ::7] = -0.0
+    elif mode == "wide":
+        # magnitudes over ~80 binades: the bracket spans far more than 256
+        # 16-bit key prefixes (the two-level search for the boundary bin)
+        S = (rng.choice([-1.0, 1.0], size=(BH, T)) *
+             np.exp(rng.uniform(-28, 28, size=(BH, T)))).astype(np.float32)
     else:
         S = (rng.standard_normal((BH, T)) * 40).astype(np.float32)
     sc = torch.from_numpy(S).cuda()
