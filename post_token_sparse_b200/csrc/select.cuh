@@ -692,6 +692,15 @@ __device__ void select_head(const SelParams& p, int bh, SelSmem& s, const KS& ks
 }
 
 // grid (ceil(T / kSelTile), BH), kSelThreads threads.
+// select_head compiled as a function of its own: with R >= 64 the streaming
+// loop's label rows fill the registers, and the selection inlined beside it
+// made the loop spill (R = 128: 676 bytes of spill loads against 8 apart).
+template <class KS>
+__device__ __noinline__ void select_head_apart(const SelParams& p, int bh, SelSmem& s,
+                                               const KS& ks) {
+  select_head(p, bh, s, ks);
+}
+
 template <int R>
 __global__ void __launch_bounds__(kSelThreads, 3)
 k_score_select(const SelParams p) {
@@ -722,7 +731,11 @@ k_score_select(const SelParams p) {
   __syncthreads();
   if (s.misc[S_LAST] == 0u) return;
   __threadfence();
-  select_head(p, bh, s, LabelKeys<R>{p.label + (size_t)bh * p.T_cap * R, s.qs});
+  const LabelKeys<R> ks{p.label + (size_t)bh * p.T_cap * R, s.qs};
+  if constexpr (R >= 64)
+    select_head_apart(p, bh, s, ks);  // keeps the wide streaming loop's registers
+  else
+    select_head(p, bh, s, ks);
   if (threadIdx.x == 0) p.arrivals[bh] = 0u;  // zero again for the next call
 }
 
