@@ -229,16 +229,15 @@ __device__ __forceinline__ uint32_t blk_select16(KeyOf key_of, int n, uint32_t r
   return (b1 << 8) | misc[S_BIN];
 }
 
-// Calls f(j, prefix) for j = 0 .. per-1 of this thread's run (j: the token's
-// offset in the run), eight prefixes per 16-byte load, read around L1 (the
-// prefixes were written by other CTAs).  The loads go out in batches of four
-// before any prefix is used: while the SM's other CTAs stream, an L2 round trip
-// takes about a microsecond, and f's shared-memory stores would otherwise keep
-// each load behind the previous word's work.
+// Prefix words a thread loads before using any: while the SM's other CTAs
+// stream, an L2 round trip takes about a microsecond, and the callers'
+// shared-memory stores would otherwise keep each load behind the previous
+// word's work.  Eight spill registers where the label rows are wide.
 constexpr int kRunBatch = 4;
 
-// Calls f(i, w) for each 16-byte word i = 0 .. per/8-1 of this thread's run: w
-// holds the prefixes of tokens 8i .. 8i+7, two a word, the lower token low.
+// Calls f(i, w) for each 16-byte word i = 0 .. per/8-1 of this thread's run,
+// read around L1 (the prefixes were written by other CTAs): w holds the
+// prefixes of tokens 8i .. 8i+7, two a word, the lower token low.
 template <class F>
 __device__ __forceinline__ void for_my_words(const uint16_t* pref, int per, F&& f) {
   const uint4* p4 = reinterpret_cast<const uint4*>(pref);
@@ -262,6 +261,8 @@ __device__ __forceinline__ void for_my_words(const uint16_t* pref, int per, F&& 
   }
 }
 
+// Calls f(j, prefix) for j = 0 .. per-1 of this thread's run (j: the token's
+// offset in the run).
 template <class F>
 __device__ __forceinline__ void for_my_run(const uint16_t* pref, int per, F&& f) {
   for_my_words(pref, per, [&](int i, const uint32_t (&w)[4]) {
